@@ -1,0 +1,156 @@
+"""Seeded synthetic inputs for MLA latent-KV decode.
+
+This module only draws inputs; it holds none of the decode arithmetic, so both
+the CUDA path (through the tests and ``bench.py``) and the float64 oracle can
+consume what it makes. Nothing here is a dataset: the shapes follow the
+DeepSeek-V2-Lite (16 heads) and V3 (128 heads) attention dimensions — a
+512-wide latent plus a 64-wide RoPE key per cached token ("DeepSeek-V2-Lite
+模型结构详解", section "五、MLA：注意力"; "深度解读DeepSeek：源码解读 DeepSeek-V3",
+section "MLA") — with random values.
+
+Draw order for one workload, all from one ``torch.Generator``:
+lengths → block table → cache pages → queries → sparse indices.
+"""
+
+from __future__ import annotations
+
+import dataclasses
+import math
+from typing import Optional, Sequence
+
+import torch
+
+PAGE = 64
+D_QK = 576
+D_LATENT = 512
+
+
+@dataclasses.dataclass(frozen=True)
+class Workload:
+    key: str
+    name: str
+    batch: int
+    q_len: int
+    heads: int
+    len_lo: int
+    len_hi: int
+    topk: int = 0
+    causal: bool = False
+    q_std: float = 1.0
+    cache_std: float = 1.0
+    seed: int = 0
+    contiguous: bool = False
+
+    @property
+    def sparse(self) -> bool:
+        return self.topk > 0
+
+
+WORKLOADS = {
+    "C1": Workload("C1", "v2lite-b1-h16-len256-contiguous", 1, 1, 16, 256, 256, seed=0, contiguous=True),
+    "C2": Workload("C2", "v2lite-b32-h16-len4096-paged", 32, 1, 16, 4096, 4096, seed=1),
+    "C3": Workload("C3", "v3-b64-h128-len1k-32k-ragged", 64, 1, 128, 1024, 32768, cache_std=0.5, seed=2),
+    "C4": Workload("C4", "v3-mtp-b32-sq2-h128-len4k-64k-causal", 32, 2, 128, 4096, 65536, causal=True, seed=3),
+    "C5": Workload("C5", "v32-sparse-b16-h128-len128k-top2048", 16, 1, 128, 131072, 131072, topk=2048, seed=4),
+}
+
+
+def make_inputs(w: Workload | str, *, seed: Optional[int] = None, lens: Optional[Sequence[int]] = None,
+                slack_pages: int = 4, nan_slack: bool = True, nan_tail: bool = False,
+                shuffle: Optional[bool] = None, chunk_pages: int = 512) -> dict:
+    """Draw one workload's inputs on the CPU.
+
+    * ``lens``: explicit per-sequence lengths (overrides the workload's range).
+    * ``slack_pages``: extra physical pages no sequence owns; filled with NaN
+      when ``nan_slack`` so that reading a wrong page poisons the result.
+    * ``nan_tail``: fill the unused slots of each sequence's last page with NaN
+      (they sit inside owned pages and must be masked, never summed).
+    * ``shuffle``: random physical page order (default: not for contiguous workloads).
+
+    Returns a dict with ``q [B,Sq,H,576] bf16``, ``cache [P,64,576] bf16``,
+    ``block_table [B,maxp] int32`` (-1 past each sequence's pages),
+    ``seq_lens [B] int32``, ``indices [B,Sq,topk] int32`` or None, and the
+    workload fields.
+    """
+    if isinstance(w, str):
+        w = WORKLOADS[w]
+    g = torch.Generator().manual_seed(w.seed if seed is None else seed)
+    B = w.batch
+    if lens is not None:
+        seq_lens = torch.as_tensor(list(lens), dtype=torch.int64)
+        assert seq_lens.numel() == B
+    elif w.len_lo == w.len_hi:
+        seq_lens = torch.full((B,), w.len_lo, dtype=torch.int64)
+    else:
+        seq_lens = torch.randint(w.len_lo, w.len_hi + 1, (B,), generator=g, dtype=torch.int64)
+    pages_per_seq = (seq_lens + PAGE - 1) // PAGE
+    used = int(pages_per_seq.sum())
+    num_pages = max(used + slack_pages, 1)
+    maxp = max(int(pages_per_seq.max()) if B > 0 else 0, 1)
+
+    do_shuffle = (not w.contiguous) if shuffle is None else shuffle
+    order = torch.randperm(used, generator=g) if do_shuffle else torch.arange(used)
+    block_table = torch.full((B, maxp), -1, dtype=torch.int32)
+    pos = 0
+    for b in range(B):
+        n = int(pages_per_seq[b])
+        block_table[b, :n] = order[pos:pos + n].to(torch.int32)
+        pos += n
+
+    cache = torch.empty((num_pages, PAGE, D_QK), dtype=torch.bfloat16)
+    for p0 in range(0, used, chunk_pages):
+        p1 = min(p0 + chunk_pages, used)
+        blk = torch.randn((p1 - p0, PAGE, D_QK), generator=g, dtype=torch.float32)
+        if w.cache_std != 1.0:
+            blk.mul_(w.cache_std)
+        cache[p0:p1] = blk.to(torch.bfloat16)
+    if used < num_pages:
+        cache[used:] = float("nan") if nan_slack else 0.0
+    if nan_tail:
+        for b in range(B):
+            L = int(seq_lens[b])
+            if L % PAGE and L > 0:
+                last = int(block_table[b, (L - 1) // PAGE])
+                cache[last, L % PAGE:] = float("nan")
+
+    q = torch.randn((B, w.q_len, w.heads, D_QK), generator=g, dtype=torch.float32)
+    if w.q_std != 1.0:
+        q.mul_(w.q_std)
+    q = q.to(torch.bfloat16)
+
+    indices = None
+    if w.topk > 0:
+        indices = torch.empty((B, w.q_len, w.topk), dtype=torch.int32)
+        for b in range(B):
+            for i in range(w.q_len):
+                L = int(seq_lens[b])
+                perm = torch.randperm(L, generator=g)[: w.topk]
+                row = torch.full((w.topk,), -1, dtype=torch.int32)
+                row[: perm.numel()] = perm.to(torch.int32)
+                indices[b, i] = row
+
+    return {
+        "workload": w,
+        "q": q,
+        "cache": cache,
+        "block_table": block_table,
+        "seq_lens": seq_lens.to(torch.int32),
+        "indices": indices,
+        "batch": B,
+        "q_len": w.q_len,
+        "heads": w.heads,
+        "topk": w.topk,
+        "causal": w.causal,
+        "num_pages": num_pages,
+        "max_pages_per_seq": maxp,
+    }
+
+
+def small(key: str = "t", *, batch: int, heads: int, q_len: int = 1, lens: Sequence[int], topk: int = 0,
+          causal: bool = False, seed: int = 0, q_std: float = 1.0, cache_std: float = 1.0,
+          **kw) -> dict:
+    """A custom (usually small) workload with explicit lengths."""
+    w = Workload(key, f"custom-b{batch}-h{heads}-sq{q_len}", batch, q_len, heads, min(lens), max(lens), topk=topk,
+                 causal=causal, q_std=q_std, cache_std=cache_std, seed=seed)
+    return make_inputs(w, lens=lens, **kw)
+
