@@ -1,0 +1,149 @@
+/*
+ * libmla — MLA (multi-head latent attention) decode over a paged latent KV
+ * cache, for NVIDIA B200 (sm_100a).
+ *
+ * What one decode step computes (for every sequence b, query token i, head h):
+ *
+ *   T      = visible cache positions of (b, i): dense t < L_b, or
+ *            t <= L_b - Sq + i when causal, or the listed top-k positions
+ *   row(t) = kv_cache[block_table[b][t / 64]][t % 64][0:576]  (c_kv[512] || k_pe[64])
+ *   s_t    = scale * ( q[b,i,h,0:512] . row(t)[0:512] + q[b,i,h,512:576] . row(t)[512:576] )
+ *   lse    = ln sum_t exp(s_t)
+ *   out    = sum_t exp(s_t - lse) * row(t)[0:512]
+ *
+ * This is the absorbed branch of DeepSeek's MLA as printed in
+ * "深度解读DeepSeek：源码解读 DeepSeek-V3", section "MLA" (two-term score
+ * against kv_cache and pe_cache, float32 softmax, latent PV), with W_UK
+ * folded into q and W_UV left to the caller ("DeepSeek-V2-Lite 模型结构详解",
+ * section "五、MLA：注意力", the two absorption identities). The scale is
+ * 1/sqrt(192): a query/key head is 128 content + 64 RoPE dimensions (same
+ * page, "为什么 Q/K 是 192 维而 V 只有 128 维").
+ *
+ * Calling sequence, all asynchronous on one stream, no host synchronisation
+ * (so it can be captured in a CUDA graph):
+ *
+ *   mla_decode_plan  -> split schedule from device seq_lens
+ *   mla_decode       -> attention; unsplit rows final, split rows as partials
+ *   mla_combine      -> LSE merge of partials into out / lse
+ *
+ * Ownership: the caller owns every buffer (plan, workspace, inputs, outputs).
+ * The library allocates no device memory and keeps no state between calls
+ * beyond per-device launch attributes. Pointers are device pointers unless
+ * stated otherwise. q, kv_cache and out must be 16-byte aligned and densely
+ * packed row-major with the shapes given below.
+ *
+ * Errors: argument problems are reported synchronously, before any launch,
+ * as MLA_ERR_INVALID_ARG / MLA_ERR_UNSUPPORTED / MLA_ERR_WORKSPACE_TOO_SMALL;
+ * launch failures as MLA_ERR_CUDA. Problems only visible on the device
+ * (a length beyond the block table, a page id outside the cache, a sparse
+ * index outside [0, L_b)) never trap: the offending tokens are skipped
+ * (rows attend to the remaining tokens; a row left with none gets out = 0,
+ * lse = -inf) and a bit is set in the plan's error word, read by
+ * mla_get_error. Every pipeline wait inside the kernels is bounded; a wait
+ * that runs out sets MLA_DEVERR_TIMEOUT and the kernel returns.
+ */
+#ifndef LIBMLA_MLA_H_
+#define LIBMLA_MLA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MLA_API __attribute__((visibility("default")))
+#else
+#define MLA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A cudaStream_t (NULL = legacy default stream). */
+typedef struct CUstream_st* mla_stream_t;
+
+typedef enum {
+  MLA_OK = 0,
+  MLA_ERR_INVALID_ARG = 1,         /* NULL / misaligned pointer, negative size, bad flag */
+  MLA_ERR_UNSUPPORTED = 2,         /* valid but not implemented (e.g. H > 128, d_latent != 512) */
+  MLA_ERR_WORKSPACE_TOO_SMALL = 3, /* plan or workspace buffer smaller than the sizing query says */
+  MLA_ERR_CUDA = 4,                /* a CUDA runtime/driver call failed */
+  MLA_ERR_DEVICE_BOUNDS = 5,       /* mla_get_error: bad length, page id or index seen on device */
+  MLA_ERR_DEVICE_TIMEOUT = 6       /* mla_get_error: a bounded device wait ran out */
+} mla_status_t;
+
+/* Bits of the device error word (mla_get_error). */
+#define MLA_DEVERR_SEQ_LEN 0x1u /* seq_lens[b] < 0 or > max_pages_per_seq * 64: sequence skipped */
+#define MLA_DEVERR_PAGE_ID 0x2u /* block_table entry outside [0, num_pages): that page skipped */
+#define MLA_DEVERR_INDEX 0x4u   /* sparse index outside [-1, L_b): that index skipped */
+#define MLA_DEVERR_TIMEOUT 0x8u /* a pipeline wait ran out: results are invalid */
+
+typedef struct {
+  int32_t batch;             /* B >= 0 */
+  int32_t q_len;             /* Sq >= 1: new query tokens per sequence (2 = MTP pair) */
+  int32_t num_heads;         /* H: multiple of 16, 16..128 */
+  int32_t d_latent;          /* must be 512 (kv_lora_rank) */
+  int32_t d_rope;            /* must be 64 (qk_rope_head_dim) */
+  int32_t page_size;         /* must be 64 tokens */
+  int32_t num_pages;         /* physical pages in kv_cache, >= 1 */
+  int32_t max_pages_per_seq; /* block_table row stride (entries), >= 1 */
+  int32_t topk;              /* 0: dense; > 0: sparse, topk indices per (b, i) */
+  int32_t causal;            /* dense only: 1 = query i sees t <= L_b - Sq + i */
+  float softmax_scale;       /* > 0; 1/sqrt(192) for DeepSeek V2/V3 */
+  int32_t num_sms;           /* SMs to spread the work over; 0 = all SMs of the current device */
+} mla_decode_desc_t;
+
+/* Bytes of the plan buffer for this descriptor (0 if the descriptor is invalid).
+ * The plan holds a small header, per-task page prefix sums and token counts,
+ * and the device error word. */
+MLA_API size_t mla_plan_bytes(const mla_decode_desc_t* desc);
+
+/* Bytes of the workspace: fp32 partial outputs and LSEs for the worst-case
+ * number of splits (one slot per (worker, task) overlap), so that no host
+ * synchronisation is needed to size it (0 if the descriptor is invalid). */
+MLA_API size_t mla_workspace_bytes(const mla_decode_desc_t* desc);
+
+/* Number of 2-CTA workers (clusters) the decode kernel runs on the current
+ * device for this descriptor (0 if invalid). Plan, decode and combine must
+ * see the same value, i.e. the same device and desc->num_sms. */
+MLA_API int32_t mla_num_workers(const mla_decode_desc_t* desc);
+
+/* Step a1: split schedule. seq_lens: device int32 [B] (tokens cached per
+ * sequence, including the Sq new ones). Writes the plan (device buffer of at
+ * least mla_plan_bytes) and clears its error word. One small kernel. */
+MLA_API mla_status_t mla_decode_plan(const mla_decode_desc_t* desc, const int32_t* seq_lens, void* plan,
+                             size_t plan_bytes, mla_stream_t stream);
+
+/* Steps a2-a7: attention over the latent cache.
+ *   q            bf16 [B, Sq, H, 576]  absorbed queries (q_lat[512] || q_pe[64])
+ *   kv_cache     bf16 [num_pages, 64, 576]  (c_kv[512] || k_pe[64] per token)
+ *   block_table  int32 [B, max_pages_per_seq]  page ids of each sequence, in order
+ *   seq_lens     int32 [B]  (the array given to mla_decode_plan)
+ *   topk_indices int32 [B, Sq, topk] logical positions in [0, L_b), -1 = skip;
+ *                NULL when desc->topk == 0
+ *   out          bf16 [B, Sq, H, 512]   lse  fp32 [B, Sq, H] (natural log)
+ *   workspace    at least mla_workspace_bytes
+ * Rows whose task is not split are final after this call; the others are
+ * final after mla_combine. */
+MLA_API mla_status_t mla_decode(const mla_decode_desc_t* desc, void* plan, const void* q, const void* kv_cache,
+                        const int32_t* block_table, const int32_t* seq_lens, const int32_t* topk_indices,
+                        void* out, float* lse, void* workspace, size_t workspace_bytes, mla_stream_t stream);
+
+/* Step a8: merge split partials by LSE (lse = ln sum_i exp(lse_i),
+ * out = sum_i exp(lse_i - lse) out_i) and write empty rows as out = 0,
+ * lse = -inf. Must follow mla_decode on the same stream. */
+MLA_API mla_status_t mla_combine(const mla_decode_desc_t* desc, void* plan, const void* workspace, size_t workspace_bytes,
+                         void* out, float* lse, mla_stream_t stream);
+
+/* Synchronises the stream, reads the plan's device error word into
+ * *error_bits (may be NULL) and maps it to MLA_OK, MLA_ERR_DEVICE_TIMEOUT
+ * (timeout bit set) or MLA_ERR_DEVICE_BOUNDS (any other bit). */
+MLA_API mla_status_t mla_get_error(const void* plan, uint32_t* error_bits, mla_stream_t stream);
+
+/* Static string for a status code. */
+MLA_API const char* mla_status_string(mla_status_t status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LIBMLA_MLA_H_ */

@@ -1,0 +1,154 @@
+"""ctypes binding of ``libmla.so`` (include/mla.h): the same names, argument
+marshalling only. Every step of the decode runs in the library's CUDA
+kernels; there is no fallback. Importing this module without the built
+library raises ``RuntimeError``.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmla.so")
+
+MLA_OK = 0
+MLA_ERR_INVALID_ARG = 1
+MLA_ERR_UNSUPPORTED = 2
+MLA_ERR_WORKSPACE_TOO_SMALL = 3
+MLA_ERR_CUDA = 4
+MLA_ERR_DEVICE_BOUNDS = 5
+MLA_ERR_DEVICE_TIMEOUT = 6
+
+MLA_DEVERR_SEQ_LEN = 0x1
+MLA_DEVERR_PAGE_ID = 0x2
+MLA_DEVERR_INDEX = 0x4
+MLA_DEVERR_TIMEOUT = 0x8
+
+EXPORTED = (
+    "mla_plan_bytes", "mla_workspace_bytes", "mla_num_workers", "mla_decode_plan", "mla_decode",
+    "mla_combine", "mla_get_error", "mla_status_string",
+)
+
+DEFAULT_SOFTMAX_SCALE = 1.0 / math.sqrt(192.0)
+
+
+class mla_decode_desc_t(ctypes.Structure):
+    _fields_ = [
+        ("batch", ctypes.c_int32),
+        ("q_len", ctypes.c_int32),
+        ("num_heads", ctypes.c_int32),
+        ("d_latent", ctypes.c_int32),
+        ("d_rope", ctypes.c_int32),
+        ("page_size", ctypes.c_int32),
+        ("num_pages", ctypes.c_int32),
+        ("max_pages_per_seq", ctypes.c_int32),
+        ("topk", ctypes.c_int32),
+        ("causal", ctypes.c_int32),
+        ("softmax_scale", ctypes.c_float),
+        ("num_sms", ctypes.c_int32),
+    ]
+
+
+def make_desc(*, batch: int, q_len: int, num_heads: int, num_pages: int, max_pages_per_seq: int, topk: int = 0,
+              causal: bool = False, softmax_scale: float = DEFAULT_SOFTMAX_SCALE, num_sms: int = 0,
+              d_latent: int = 512, d_rope: int = 64, page_size: int = 64) -> mla_decode_desc_t:
+    return mla_decode_desc_t(batch, q_len, num_heads, d_latent, d_rope, page_size, num_pages, max_pages_per_seq,
+                             topk, int(bool(causal)), softmax_scale, num_sms)
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(
+            f"libmla.so is not built ({LIB_PATH} missing): run `python -m mla_latent_kv_26_b200.build` "
+            "(there is no non-CUDA fallback)")
+    lib = ctypes.CDLL(LIB_PATH)
+    P = ctypes.c_void_p
+    D = ctypes.POINTER(mla_decode_desc_t)
+    sig = {
+        "mla_plan_bytes": (ctypes.c_size_t, [D]),
+        "mla_workspace_bytes": (ctypes.c_size_t, [D]),
+        "mla_num_workers": (ctypes.c_int32, [D]),
+        "mla_decode_plan": (ctypes.c_int, [D, P, P, ctypes.c_size_t, P]),
+        "mla_decode": (ctypes.c_int, [D, P, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]),
+        "mla_combine": (ctypes.c_int, [D, P, P, ctypes.c_size_t, P, P, P]),
+        "mla_get_error": (ctypes.c_int, [P, ctypes.POINTER(ctypes.c_uint32), P]),
+        "mla_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+_lib = _load()
+
+
+def _ptr(x) -> Optional[int]:
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def _stream(s) -> Optional[int]:
+    if s is None:
+        return None
+    if isinstance(s, int):
+        return s
+    return s.cuda_stream
+
+
+class MlaError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {mla_status_string(status)} ({status})")
+        self.status = status
+
+
+def mla_status_string(status: int) -> str:
+    return _lib.mla_status_string(int(status)).decode()
+
+
+def mla_plan_bytes(desc: mla_decode_desc_t) -> int:
+    return int(_lib.mla_plan_bytes(ctypes.byref(desc)))
+
+
+def mla_workspace_bytes(desc: mla_decode_desc_t) -> int:
+    return int(_lib.mla_workspace_bytes(ctypes.byref(desc)))
+
+
+def mla_num_workers(desc: mla_decode_desc_t) -> int:
+    return int(_lib.mla_num_workers(ctypes.byref(desc)))
+
+
+def mla_decode_plan(desc, seq_lens, plan, plan_bytes: int, stream=None) -> int:
+    return int(_lib.mla_decode_plan(ctypes.byref(desc), _ptr(seq_lens), _ptr(plan), int(plan_bytes),
+                                    _stream(stream)))
+
+
+def mla_decode(desc, plan, q, kv_cache, block_table, seq_lens, topk_indices, out, lse, workspace,
+               workspace_bytes: int, stream=None) -> int:
+    return int(_lib.mla_decode(ctypes.byref(desc), _ptr(plan), _ptr(q), _ptr(kv_cache), _ptr(block_table),
+                               _ptr(seq_lens), _ptr(topk_indices), _ptr(out), _ptr(lse), _ptr(workspace),
+                               int(workspace_bytes), _stream(stream)))
+
+
+def mla_combine(desc, plan, workspace, workspace_bytes: int, out, lse, stream=None) -> int:
+    return int(_lib.mla_combine(ctypes.byref(desc), _ptr(plan), _ptr(workspace), int(workspace_bytes), _ptr(out),
+                                _ptr(lse), _stream(stream)))
+
+
+def mla_get_error(plan, stream=None):
+    """Synchronises ``stream``; returns ``(status, error_bits)``."""
+    bits = ctypes.c_uint32(0)
+    st = int(_lib.mla_get_error(_ptr(plan), ctypes.byref(bits), _stream(stream)))
+    return st, int(bits.value)
+
+
+def check(status: int, what: str) -> None:
+    if status != MLA_OK:
+        raise MlaError(status, what)

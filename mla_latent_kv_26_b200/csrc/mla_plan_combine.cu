@@ -1,0 +1,139 @@
+// Steps a1 (split schedule) and a8 (LSE merge of split partials).
+#include <math.h>
+
+#include "common.cuh"
+
+namespace mla {
+
+// One block of 1024 threads. Task t = b * Sq + i gets ntok[t] tokens (index
+// slots when sparse) and ceil(ntok/64) pages; prefix[] lays the tasks' pages
+// end to end; worker w owns global pages [w*quota, (w+1)*quota).
+__global__ void __launch_bounds__(1024) mla_plan_kernel(PlanArgs a) {
+  __shared__ int s_scan[1024];
+  __shared__ int s_carry;
+  __shared__ unsigned s_err;
+  const int tid = threadIdx.x;
+  const int T = a.batch * a.q_len;
+  int32_t* prefix = a.plan + plan_prefix_off();
+  int32_t* ntok = a.plan + plan_ntok_off(T);
+  if (tid == 0) {
+    s_carry = 0;
+    s_err = 0u;
+  }
+  __syncthreads();
+  const long long cap = (long long)a.max_pages_per_seq * kPage;
+  for (int base = 0; base < T; base += 1024) {
+    const int t = base + tid;
+    int pages = 0;
+    if (t < T) {
+      const int b = t / a.q_len, i = t % a.q_len;
+      const int L = a.seq_lens[b];
+      const bool ok = L >= 0 && (long long)L <= cap;
+      int n = 0;
+      if (ok) n = a.topk > 0 ? a.topk : (a.causal ? max(L - a.q_len + i + 1, 0) : L);
+      else atomicOr(&s_err, kErrSeqLen);
+      ntok[t] = n;
+      pages = (n + kPage - 1) / kPage;
+    }
+    s_scan[tid] = pages;
+    __syncthreads();
+    for (int off = 1; off < 1024; off <<= 1) {
+      const int v = tid >= off ? s_scan[tid - off] : 0;
+      __syncthreads();
+      s_scan[tid] += v;
+      __syncthreads();
+    }
+    if (t < T) prefix[t] = s_carry + s_scan[tid] - pages;
+    __syncthreads();
+    if (tid == 1023) s_carry += s_scan[1023];
+    __syncthreads();
+  }
+  if (tid == 0) {
+    const int total = s_carry;
+    prefix[T] = total;
+    const int quota = max(1, (total + a.workers - 1) / a.workers);
+    a.plan[kPlanErr] = (int32_t)s_err;
+    a.plan[kPlanTasks] = T;
+    a.plan[kPlanQuota] = quota;
+    a.plan[kPlanTotal] = total;
+    a.plan[kPlanWorkers] = a.workers;
+    a.plan[kPlanHeads] = a.heads;
+    a.plan[6] = 0;
+    a.plan[7] = 0;
+  }
+}
+
+// grid (T, ceil(H/8)), 256 threads: one warp per (task, head) row.
+// Unsplit tasks were finished by the decode kernel; empty tasks get out = 0,
+// lse = -inf; split tasks merge their partials (slot = worker + task):
+// lse = M + ln sum_w exp(lse_w - M), out = sum_w exp(lse_w - lse) * o_w.
+__global__ void __launch_bounds__(256) mla_combine_kernel(CombineArgs a) {
+  const int T = a.plan[kPlanTasks];
+  const int quota = a.plan[kPlanQuota];
+  const int t = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int h = blockIdx.y * 8 + warp;
+  if (t >= T || h >= a.heads) return;
+  const int32_t* prefix = a.plan + plan_prefix_off();
+  const int p0 = prefix[t], p1 = prefix[t + 1];
+  const size_t row = (size_t)t * a.heads + h;
+  __nv_bfloat16* orow = a.out + row * kDLatent;
+  const int w0 = p0 / quota;
+  const int w1 = p1 > p0 ? (p1 - 1) / quota : w0;
+  if (p1 > p0 && w0 == w1) return;
+
+  float m = -INFINITY;
+  if (p1 > p0) {
+    for (int w = w0; w <= w1; ++w) m = fmaxf(m, a.part_lse[(size_t)(w + t) * a.heads + h]);
+  }
+  if (m == -INFINITY) {
+    const __nv_bfloat162 z = __floats2bfloat162_rn(0.f, 0.f);
+    for (int j = 0; j < 4; ++j) {
+      __nv_bfloat162* dst = reinterpret_cast<__nv_bfloat162*>(orow + lane * 4 + 128 * j);
+      dst[0] = z;
+      dst[1] = z;
+    }
+    if (lane == 0) a.lse[row] = -INFINITY;
+    return;
+  }
+  float acc[16];
+#pragma unroll
+  for (int j = 0; j < 16; ++j) acc[j] = 0.f;
+  float sum = 0.f;
+  for (int w = w0; w <= w1; ++w) {
+    const size_t srow = (size_t)(w + t) * a.heads + h;
+    const float l = a.part_lse[srow];
+    const float e = (l == -INFINITY) ? 0.f : expf(l - m);
+    sum += e;
+    const float4* src = reinterpret_cast<const float4*>(a.part_o + srow * kDLatent);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float4 v = src[lane + 32 * j];
+      acc[4 * j + 0] += e * v.x;
+      acc[4 * j + 1] += e * v.y;
+      acc[4 * j + 2] += e * v.z;
+      acc[4 * j + 3] += e * v.w;
+    }
+  }
+  const float inv = 1.f / sum;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    __nv_bfloat162* dst = reinterpret_cast<__nv_bfloat162*>(orow + lane * 4 + 128 * j);
+    dst[0] = __floats2bfloat162_rn(acc[4 * j + 0] * inv, acc[4 * j + 1] * inv);
+    dst[1] = __floats2bfloat162_rn(acc[4 * j + 2] * inv, acc[4 * j + 3] * inv);
+  }
+  if (lane == 0) a.lse[row] = m + logf(sum);
+}
+
+cudaError_t launch_plan(const PlanArgs& args, cudaStream_t stream) {
+  mla_plan_kernel<<<1, 1024, 0, stream>>>(args);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_combine(const CombineArgs& args, int tasks, cudaStream_t stream) {
+  dim3 grid(tasks, (args.heads + 7) / 8);
+  mla_combine_kernel<<<grid, 256, 0, stream>>>(args);
+  return cudaGetLastError();
+}
+
+}  // namespace mla

@@ -1,0 +1,85 @@
+"""Torch-facing wrapper around the C ABI: owns the plan / workspace / output
+buffers for one decode shape and issues the three library calls on a CUDA
+stream. It checks tensor dtypes, shapes and devices and passes raw pointers;
+all arithmetic happens in libmla's kernels.
+"""
+
+from __future__ import annotations
+
+from typing import Optional
+
+import torch
+
+from . import binding as B
+
+
+class MlaDecoder:
+    def __init__(self, *, batch: int, q_len: int, num_heads: int, num_pages: int, max_pages_per_seq: int,
+                 topk: int = 0, causal: bool = False, softmax_scale: float = B.DEFAULT_SOFTMAX_SCALE,
+                 num_sms: int = 0, device="cuda"):
+        self.desc = B.make_desc(batch=batch, q_len=q_len, num_heads=num_heads, num_pages=num_pages,
+                                max_pages_per_seq=max_pages_per_seq, topk=topk, causal=causal,
+                                softmax_scale=softmax_scale, num_sms=num_sms)
+        dev = torch.device(device)
+        if dev.type == "cuda" and dev.index is None:
+            dev = torch.device("cuda", torch.cuda.current_device())
+        self.device = dev
+        with torch.cuda.device(self.device):
+            self.plan_bytes = B.mla_plan_bytes(self.desc)
+            self.workspace_bytes = B.mla_workspace_bytes(self.desc)
+            self.num_workers = B.mla_num_workers(self.desc)
+        if self.plan_bytes == 0 or self.workspace_bytes == 0:
+            raise B.MlaError(B.MLA_ERR_INVALID_ARG, "descriptor rejected by the sizing queries")
+        self.plan = torch.empty(self.plan_bytes, dtype=torch.uint8, device=self.device)
+        self.workspace = torch.empty(self.workspace_bytes, dtype=torch.uint8, device=self.device)
+        self.out = torch.empty(batch, q_len, num_heads, 512, dtype=torch.bfloat16, device=self.device)
+        self.lse = torch.empty(batch, q_len, num_heads, dtype=torch.float32, device=self.device)
+
+    def _stream(self, stream):
+        return torch.cuda.current_stream(self.device) if stream is None else stream
+
+    def _check(self, name, t, dtype, shape=None):
+        if t.device != self.device or t.dtype != dtype or not t.is_contiguous():
+            raise ValueError(f"{name}: need a contiguous {dtype} tensor on {self.device}")
+        if shape is not None and tuple(t.shape) != tuple(shape):
+            raise ValueError(f"{name}: shape {tuple(t.shape)} != {tuple(shape)}")
+
+    def plan_step(self, seq_lens: torch.Tensor, stream=None) -> None:
+        d = self.desc
+        self._check("seq_lens", seq_lens, torch.int32, (d.batch,))
+        B.check(B.mla_decode_plan(d, seq_lens, self.plan, self.plan_bytes, self._stream(stream)), "mla_decode_plan")
+
+    def decode_step(self, q, kv_cache, block_table, seq_lens, indices: Optional[torch.Tensor] = None,
+                    stream=None) -> None:
+        d = self.desc
+        self._check("q", q, torch.bfloat16, (d.batch, d.q_len, d.num_heads, 576))
+        self._check("kv_cache", kv_cache, torch.bfloat16, (d.num_pages, 64, 576))
+        self._check("block_table", block_table, torch.int32, (d.batch, d.max_pages_per_seq))
+        self._check("seq_lens", seq_lens, torch.int32, (d.batch,))
+        if d.topk > 0:
+            self._check("indices", indices, torch.int32, (d.batch, d.q_len, d.topk))
+        elif indices is not None:
+            raise ValueError("indices given for a dense descriptor")
+        B.check(B.mla_decode(d, self.plan, q, kv_cache, block_table, seq_lens, indices, self.out, self.lse,
+                             self.workspace, self.workspace_bytes, self._stream(stream)), "mla_decode")
+
+    def combine_step(self, stream=None) -> None:
+        B.check(B.mla_combine(self.desc, self.plan, self.workspace, self.workspace_bytes, self.out, self.lse,
+                              self._stream(stream)), "mla_combine")
+
+    def __call__(self, q, kv_cache, block_table, seq_lens, indices=None, stream=None):
+        self.plan_step(seq_lens, stream)
+        self.decode_step(q, kv_cache, block_table, seq_lens, indices, stream)
+        self.combine_step(stream)
+        return self.out, self.lse
+
+    def error(self, stream=None):
+        """(status, device error bits); synchronises the stream."""
+        return B.mla_get_error(self.plan, self._stream(stream))
+
+
+def decoder_for(inputs: dict, *, num_sms: int = 0, device="cuda", **kw) -> MlaDecoder:
+    """An MlaDecoder sized for a dict made by ``workloads.make_inputs``."""
+    return MlaDecoder(batch=inputs["batch"], q_len=inputs["q_len"], num_heads=inputs["heads"],
+                      num_pages=inputs["num_pages"], max_pages_per_seq=inputs["max_pages_per_seq"],
+                      topk=inputs["topk"], causal=inputs["causal"], num_sms=num_sms, device=device, **kw)
