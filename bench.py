@@ -1,0 +1,423 @@
+"""Throughput of MLA latent-KV decode on B200: one step = mla_decode_plan +
+mla_decode + mla_combine over one batch of the workload (default: V3 shapes,
+B=64, H=128, ragged KV lengths 1k-32k).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload C3] [--impl reference]
+
+Prints one JSON line (rank 0). Under torchrun (N > 1) every rank decodes its
+own copy of the batch (replicas: the path has no cross-GPU exchange), so the
+job's KV-tokens/s is N x the batch over the slowest rank's time.
+
+The CPU float64 oracle is timed here as a reported baseline (``cpu_baseline``
+and ``--impl reference``) on a bounded sample of the same workload.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from mla_latent_kv_26_b200.workloads import WORKLOADS, make_inputs  # noqa: E402
+
+METRIC = "MLA decode KV-tokens/s and achieved TB/s / TFLOP/s as fraction of roofline"
+UNIT = "KV-tokens/s"
+BYTES_PER_TOKEN = 576 * 2       # one cached row: c_kv[512] + k_pe[64], bf16
+FLOPS_PER_ROW_TOKEN = 2 * (576 + 512)  # QK^T over 576 + PV over 512, multiply-add = 2
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+DECODE_SRC = os.path.join(ROOT, "mla_latent_kv_26_b200", "csrc", "mla_decode.cu")
+
+
+# ---------------------------------------------------------------- accounting
+
+
+def accounting(inp: dict) -> dict:
+    """Algorithmic work of one step (no split partials, no re-reads)."""
+    lens = [int(x) for x in inp["seq_lens"]]
+    B, Sq, H, topk = inp["batch"], inp["q_len"], inp["heads"], inp["topk"]
+    kv_tokens = 0          # distinct cache rows read per sequence
+    row_tokens = 0         # sum over (b, i) of visible tokens; x H for score rows
+    table_bytes = 0
+    for b, L in enumerate(lens):
+        if topk > 0:
+            idx = inp["indices"][b]
+            uniq = int(torch.unique(idx[idx >= 0]).numel())
+            kv_tokens += uniq
+            row_tokens += int((idx >= 0).sum())
+            table_bytes += idx.numel() * 4 + uniq * 4
+        else:
+            per_q = [max(L - Sq + i + 1, 0) if inp["causal"] else L for i in range(Sq)]
+            kv_tokens += max(per_q) if per_q else 0
+            row_tokens += sum(per_q)
+            table_bytes += ((max(per_q) + 63) // 64) * 4
+    rows = B * Sq * H
+    bytes_ = kv_tokens * BYTES_PER_TOKEN + rows * 576 * 2 + rows * 512 * 2 + rows * 4 + table_bytes + B * 4
+    flops = row_tokens * H * FLOPS_PER_ROW_TOKEN
+    return {"kv_tokens": kv_tokens, "row_tokens": row_tokens, "bytes": bytes_, "flops": flops,
+            "h2d_bytes": rows * 576 * 2 + inp["block_table"].numel() * 4 + B * 4 +
+            (inp["indices"].numel() * 4 if inp["indices"] is not None else 0),
+            "d2h_bytes": rows * 512 * 2 + rows * 4}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {k: float(p[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def decode_source_sha() -> str:
+    h = hashlib.sha256()
+    for f in ("mla_decode.cu", "sm100.cuh", "common.cuh"):
+        with open(os.path.join(ROOT, "mla_latent_kv_26_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload: str):
+    """DRAM bytes per decode launch from the committed ncu summary, if it was
+    taken on the current kernel source; else None."""
+    path = os.path.join(ROOT, "profiles", f"mla_decode_kernel_{workload}.md")
+    try:
+        text = open(path).read()
+    except OSError:
+        return None
+    m_sha = re.search(r"source_sha:\s*([0-9a-f]+)", text)
+    m_b = re.search(r"dram_bytes_per_launch:\s*([0-9]+)", text)
+    if not m_sha or not m_b or m_sha.group(1) != decode_source_sha():
+        return None
+    return int(m_b.group(1))
+
+
+# ---------------------------------------------------------------- clocks
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while running."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+               0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+    def __init__(self, device: int, interval_s: float = 0.01):
+        self.samples = []
+        self.reasons = 0
+        self.max_mhz = None
+        self.error = None
+        self._stop = threading.Event()
+        self._thread = None
+        self.interval = interval_s
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            uuid = str(torch.cuda.get_device_properties(device).uuid)
+            try:
+                self.h = pynvml.nvmlDeviceGetHandleByUUID(("GPU-" + uuid) if not uuid.startswith("GPU-") else uuid)
+            except Exception:
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(device)
+            self.nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self._get_reasons = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                getattr(pynvml, "nvmlDeviceGetCurrentClocksThrottleReasons")
+        except Exception as e:  # no NVML: report it
+            self.nv = None
+            self.error = f"nvml unavailable: {e}"
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                mhz = self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM)
+                r = int(self._get_reasons(self.h))
+                self.samples.append(mhz)
+                self.reasons |= r
+            except Exception as e:
+                self.error = str(e)
+            time.sleep(self.interval)
+
+    def __enter__(self):
+        if self.nv is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0,
+                    "note": self.error or "no samples"}
+        names = [n for bit, n in self.REASONS.items() if self.reasons & bit and n != "gpu_idle"]
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz, "reasons": names,
+                "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------- CPU oracle arm
+
+
+def oracle_sample(inp: dict, budget_s: float):
+    """Time the float64 oracle on whole sequences of the batch until the budget
+    is used; returns (kv_tokens, seconds, sequences)."""
+    import oracle
+
+    t0 = time.perf_counter()
+    toks, done = 0, 0
+    order = list(range(inp["batch"]))
+    for b in order:
+        oracle.mla_decode(inp["q"], inp["cache"], inp["block_table"], inp["seq_lens"], causal=inp["causal"],
+                          indices=inp["indices"], batches=[b])
+        L = int(inp["seq_lens"][b])
+        toks += min(inp["topk"], L) if inp["topk"] else L
+        done += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    return toks, time.perf_counter() - t0, done
+
+
+def run_reference(args, inp, rank):
+    if rank != 0:
+        return
+    torch.set_num_threads(os.cpu_count() or 1)
+    # each step: the oracle on a bounded slice (two sequences) of the batch
+    per_step = []
+    toks_total, secs_total = 0, 0.0
+    order = list(range(inp["batch"]))
+    for s in range(args.warmup + args.steps):
+        import oracle
+
+        bs = [order[(2 * s) % len(order)], order[(2 * s + 1) % len(order)]]
+        t0 = time.perf_counter()
+        oracle.mla_decode(inp["q"], inp["cache"], inp["block_table"], inp["seq_lens"], causal=inp["causal"],
+                          indices=inp["indices"], batches=bs)
+        dt = time.perf_counter() - t0
+        toks = sum(min(inp["topk"], int(inp["seq_lens"][b])) if inp["topk"] else int(inp["seq_lens"][b]) for b in bs)
+        if s >= args.warmup:
+            toks_total += toks
+            secs_total += dt
+            per_step.append(dt)
+    value = toks_total / secs_total if secs_total > 0 else 0.0
+    w = inp["workload"]
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs_total / max(args.steps, 1),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"{w.key} {w.name}", "batch": w.batch, "heads": w.heads, "q_len": w.q_len},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": torch.get_num_threads(), "kind": "oracle",
+                         "sample": "float64 CPU oracle, two whole sequences of the batch per step"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- GPU arm
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default="C3", choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="libmla", choices=["libmla", "reference"])
+    ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle time for cpu_baseline")
+    ap.add_argument("--profile", action="store_true", help="kernel launches only (for ncu): no e2e/oracle/clocks")
+    ap.add_argument("--num-sms", type=int, default=0)
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.gpus != world and world > 1:
+        args.gpus = world
+
+    inp = make_inputs(args.workload)
+
+    if args.impl == "reference":
+        run_reference(args, inp, rank)
+        return
+
+    import torch.distributed as dist
+
+    from mla_latent_kv_26_b200.decoder import decoder_for
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+
+    acc = accounting(inp)
+    g = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+    dec = decoder_for(inp, num_sms=args.num_sms, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev=None):
+        dec.plan_step(g["seq_lens"], stream)
+        if ev is not None:
+            ev[0].record(stream)
+        dec.decode_step(g["q"], g["cache"], g["block_table"], g["seq_lens"], g["indices"], stream)
+        if ev is not None:
+            ev[1].record(stream)
+        dec.combine_step(stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier(device_ids=[local])
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    st, bits = dec.error(stream)
+    if st != 0:
+        raise RuntimeError(f"device error after warm-up: status {st} bits {bits:#x}")
+
+    K = args.steps
+    kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local) if not args.profile else None
+    barrier()
+    torch.cuda.synchronize(dev)
+    if sampler:
+        sampler.__enter__()
+    t_start.record(stream)
+    for i in range(K):
+        step(kev[i])
+    t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    if sampler:
+        sampler.__exit__(None, None, None)
+    barrier()
+    elapsed_ms = t_start.elapsed_time(t_end)
+    decode_ms = sum(a.elapsed_time(b) for a, b in kev) / K
+    tmax = torch.tensor([elapsed_ms, decode_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(tmax, op=dist.ReduceOp.MAX)
+    elapsed_ms, decode_ms = float(tmax[0]), float(tmax[1])
+    ms_per_step = elapsed_ms / K
+
+    if args.profile:
+        if rank == 0:
+            print(json.dumps({"profile_run": True, "ms_per_step": ms_per_step, "decode_ms": decode_ms}))
+        if world > 1:
+            dist.destroy_process_group()
+        return
+
+    # ---- end to end through the public API with pinned host buffers
+    host_in = {k: inp[k].pin_memory() for k in ("q", "block_table", "seq_lens")}
+    if inp["indices"] is not None:
+        host_in["indices"] = inp["indices"].pin_memory()
+    host_out = torch.empty(dec.out.shape, dtype=dec.out.dtype).pin_memory()
+    host_lse = torch.empty(dec.lse.shape, dtype=dec.lse.dtype).pin_memory()
+    dev_in = {k: torch.empty_like(v, device=dev) for k, v in host_in.items()}
+
+    def e2e_step():
+        for k, v in host_in.items():
+            dev_in[k].copy_(v, non_blocking=True)
+        dec.plan_step(dev_in["seq_lens"], stream)
+        dec.decode_step(dev_in["q"], g["cache"], dev_in["block_table"], dev_in["seq_lens"], dev_in.get("indices"),
+                        stream)
+        dec.combine_step(stream)
+        host_out.copy_(dec.out, non_blocking=True)
+        host_lse.copy_(dec.lse, non_blocking=True)
+
+    for _ in range(args.warmup):
+        e2e_step()
+    K2 = max(3, min(K, 50))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    for _ in range(K2):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    e2e_ms = torch.tensor([e0.elapsed_time(e1) / K2], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
+    e2e_ms = float(e2e_ms)
+
+    st, bits = dec.error(stream)
+    if st != 0:
+        raise RuntimeError(f"device error in timed region: status {st} bits {bits:#x}")
+
+    peaks, peak_src = load_peaks()
+    t_hbm = acc["bytes"] / (peaks["hbm_gbs"] * 1e9)
+    t_tc = acc["flops"] / (peaks["bf16_tflops"] * 1e12)
+    bound = "hbm" if t_hbm >= t_tc else "tensor"
+    dec_s = decode_ms / 1e3
+    achieved_gbs = acc["bytes"] / dec_s / 1e9
+    achieved_tf = acc["flops"] / dec_s / 1e12
+    if bound == "hbm":
+        roof = {"bound": "hbm", "achieved": achieved_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved_gbs / peaks["hbm_gbs"]}
+    else:
+        roof = {"bound": "tensor", "achieved": achieved_tf, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": achieved_tf / peaks["bf16_tflops"]}
+    roof["traffic"] = profiled_traffic(args.workload)
+    roof["peak_source"] = f"{peak_src} (MEASURED_PEAKS.json burst figures)" if peak_src == "measured" else peak_src
+    roof["kernel"] = "mla_decode_kernel"
+    roof["roofline_time_us"] = max(t_hbm, t_tc) * 1e6
+    roof["kernel_time_us"] = decode_ms * 1e3
+    roof["time_frac"] = max(t_hbm, t_tc) / dec_s
+    roof["time_frac_step"] = max(t_hbm, t_tc) / (ms_per_step / 1e3)
+    roof["tb_per_s"] = achieved_gbs / 1e3
+    roof["tflop_per_s"] = achieved_tf
+    roof["tensor_frac"] = achieved_tf / peaks["bf16_tflops"]
+
+    value = world * acc["kv_tokens"] / (ms_per_step / 1e3)
+    w = inp["workload"]
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
+        "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"{w.key} {w.name}", "batch": w.batch, "q_len": w.q_len, "heads": w.heads,
+                   "kv_len": f"{w.len_lo}..{w.len_hi}" + (f" top{w.topk}" if w.topk else ""),
+                   "kv_tokens_per_step": acc["kv_tokens"], "bytes_per_step": acc["bytes"],
+                   "flops_per_step": acc["flops"], "seed": w.seed, "workers": dec.num_workers,
+                   "l2": f"inputs larger than L2 ({acc['bytes'] / 1e6:.0f} MB read per step), no flush"
+                   if acc["bytes"] > 256e6 else "inputs smaller than L2: not flushed",
+                   "parallelism": f"replicas x{world}"},
+        "roofline": roof,
+        "e2e": {"value": world * acc["kv_tokens"] / (e2e_ms / 1e3), "unit": UNIT,
+                "h2d_bytes_per_step": acc["h2d_bytes"], "d2h_bytes_per_step": acc["d2h_bytes"],
+                "ms_per_step": e2e_ms},
+        "gpu_launches": 3 * K,
+        "clocks": sampler.summary() if sampler else None,
+    }
+    if rank == 0 and world == 1:
+        torch.set_num_threads(os.cpu_count() or 1)
+        toks, secs, nseq = oracle_sample(inp, args.cpu_budget)
+        line["cpu_baseline"] = {"value": toks / secs, "unit": UNIT, "cores": torch.get_num_threads(),
+                                "kind": "oracle",
+                                "sample": f"{nseq} of {inp['batch']} sequences ({toks} KV tokens) of the same batch, "
+                                          f"float64, {secs:.1f} s"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

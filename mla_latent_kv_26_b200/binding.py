@@ -12,7 +12,7 @@ import os
 from typing import Optional
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libmla.so")
+LIB_PATH = os.environ.get("MLA_LIB", os.path.join(_HERE, "libmla.so"))
 
 MLA_OK = 0
 MLA_ERR_INVALID_ARG = 1

@@ -41,7 +41,7 @@ struct DecodeArgs {
   __nv_bfloat16* out;           // [B, Sq, H, 512]
   float* lse;                   // [B, Sq, H]
   float* part_o;                // [slots, H, 512]
-  float* part_lse;              // [slots, H]
+  float* part_lse;              // [slots, 2, H]
   int32_t* plan;
   int batch, q_len, heads, num_pages, max_pages_per_seq, topk;
   float scale_log2;             // softmax_scale * log2(e)
@@ -49,7 +49,7 @@ struct DecodeArgs {
 
 struct CombineArgs {
   const float* part_o;
-  const float* part_lse;
+  const float* part_lse;  // [slots, 2, H]
   const int32_t* plan;
   __nv_bfloat16* out;
   float* lse;
@@ -60,8 +60,9 @@ struct CombineArgs {
 __host__ __device__ inline size_t part_o_bytes(int slots, int heads) {
   return (size_t)slots * heads * kDLatent * sizeof(float);
 }
+// one LSE per (slot, CTA half, head): each half of a split row has its own normaliser
 __host__ __device__ inline size_t part_lse_bytes(int slots, int heads) {
-  return (size_t)slots * heads * sizeof(float);
+  return (size_t)slots * 2 * heads * sizeof(float);
 }
 
 }  // namespace mla

@@ -65,7 +65,9 @@ __global__ void __launch_bounds__(1024) mla_plan_kernel(PlanArgs a) {
 
 // grid (T, ceil(H/8)), 256 threads: one warp per (task, head) row.
 // Unsplit tasks were finished by the decode kernel; empty tasks get out = 0,
-// lse = -inf; split tasks merge their partials (slot = worker + task):
+// lse = -inf; split tasks merge their partials (slot = worker + task). Each
+// half of the 512 output columns was normalised on its own (one per CTA of
+// the worker), so each half merges with its own LSEs:
 // lse = M + ln sum_w exp(lse_w - M), out = sum_w exp(lse_w - lse) * o_w.
 __global__ void __launch_bounds__(256) mla_combine_kernel(CombineArgs a) {
   const int T = a.plan[kPlanTasks];
@@ -82,11 +84,14 @@ __global__ void __launch_bounds__(256) mla_combine_kernel(CombineArgs a) {
   const int w1 = p1 > p0 ? (p1 - 1) / quota : w0;
   if (p1 > p0 && w0 == w1) return;
 
-  float m = -INFINITY;
+  float m[2] = {-INFINITY, -INFINITY};
   if (p1 > p0) {
-    for (int w = w0; w <= w1; ++w) m = fmaxf(m, a.part_lse[(size_t)(w + t) * a.heads + h]);
+    for (int w = w0; w <= w1; ++w) {
+#pragma unroll
+      for (int g = 0; g < 2; ++g) m[g] = fmaxf(m[g], a.part_lse[((size_t)(w + t) * 2 + g) * a.heads + h]);
+    }
   }
-  if (m == -INFINITY) {
+  if (m[0] == -INFINITY) {
     const __nv_bfloat162 z = __floats2bfloat162_rn(0.f, 0.f);
     for (int j = 0; j < 4; ++j) {
       __nv_bfloat162* dst = reinterpret_cast<__nv_bfloat162*>(orow + lane * 4 + 128 * j);
@@ -99,30 +104,35 @@ __global__ void __launch_bounds__(256) mla_combine_kernel(CombineArgs a) {
   float acc[16];
 #pragma unroll
   for (int j = 0; j < 16; ++j) acc[j] = 0.f;
-  float sum = 0.f;
+  float sum[2] = {0.f, 0.f};
   for (int w = w0; w <= w1; ++w) {
     const size_t srow = (size_t)(w + t) * a.heads + h;
-    const float l = a.part_lse[srow];
-    const float e = (l == -INFINITY) ? 0.f : expf(l - m);
-    sum += e;
+    float e[2];
+#pragma unroll
+    for (int g = 0; g < 2; ++g) {
+      const float l = a.part_lse[((size_t)(w + t) * 2 + g) * a.heads + h];
+      e[g] = (l == -INFINITY) ? 0.f : expf(l - m[g]);
+      sum[g] += e[g];
+    }
     const float4* src = reinterpret_cast<const float4*>(a.part_o + srow * kDLatent);
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
+    for (int j = 0; j < 4; ++j) {  // columns lane*4 + 128 j: j < 2 in the first half
+      const float ej = e[j >> 1];
       const float4 v = src[lane + 32 * j];
-      acc[4 * j + 0] += e * v.x;
-      acc[4 * j + 1] += e * v.y;
-      acc[4 * j + 2] += e * v.z;
-      acc[4 * j + 3] += e * v.w;
+      acc[4 * j + 0] += ej * v.x;
+      acc[4 * j + 1] += ej * v.y;
+      acc[4 * j + 2] += ej * v.z;
+      acc[4 * j + 3] += ej * v.w;
     }
   }
-  const float inv = 1.f / sum;
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
+    const float inv = 1.f / sum[j >> 1];
     __nv_bfloat162* dst = reinterpret_cast<__nv_bfloat162*>(orow + lane * 4 + 128 * j);
     dst[0] = __floats2bfloat162_rn(acc[4 * j + 0] * inv, acc[4 * j + 1] * inv);
     dst[1] = __floats2bfloat162_rn(acc[4 * j + 2] * inv, acc[4 * j + 3] * inv);
   }
-  if (lane == 0) a.lse[row] = m + logf(sum);
+  if (lane == 0) a.lse[row] = m[0] + logf(sum[0]);
 }
 
 cudaError_t launch_plan(const PlanArgs& args, cudaStream_t stream) {

@@ -132,6 +132,14 @@ MLA_DEV void st_async_v4(uint32_t cluster_addr, uint32_t a, uint32_t b, uint32_t
                : "memory");
 }
 
+// 4-byte asynchronous store into another CTA's shared memory; completes 4
+// bytes on that CTA's barrier.
+MLA_DEV void st_async_b32(uint32_t cluster_addr, uint32_t v, uint32_t cluster_bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];" ::"r"(cluster_addr), "r"(v),
+               "r"(cluster_bar)
+               : "memory");
+}
+
 MLA_DEV uint4 ld_shared_v4(uint32_t addr) {
   uint4 v;
   asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
@@ -199,6 +207,13 @@ MLA_DEV void tmem_ld_32(uint32_t taddr, uint32_t (&r)[32]) {
         "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
       : "r"(taddr));
 }
+MLA_DEV void tmem_ld_16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
 MLA_DEV void tmem_st_32(uint32_t taddr, const uint32_t (&r)[32]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
@@ -230,6 +245,22 @@ MLA_DEV float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// 24-bit floats: an fp32 bit pattern rounded (half up in magnitude) to its
+// top three bytes (sign, exponent, 15 mantissa bits; relative error <= 2^-16).
+// Four of them pack into three words, byte-wise little endian.
+MLA_DEV void pack24x4(const uint32_t* f, uint32_t* w) {
+  const uint32_t r0 = f[0] + 0x80u, r1 = f[1] + 0x80u, r2 = f[2] + 0x80u, r3 = f[3] + 0x80u;
+  w[0] = __byte_perm(r0, r1, 0x5321);  // r0.b1 r0.b2 r0.b3 r1.b1
+  w[1] = __byte_perm(r1, r2, 0x6532);  // r1.b2 r1.b3 r2.b1 r2.b2
+  w[2] = __byte_perm(r2, r3, 0x7653);  // r2.b3 r3.b1 r3.b2 r3.b3
+}
+MLA_DEV void unpack24x4(uint32_t w0, uint32_t w1, uint32_t w2, float* f) {
+  f[0] = __uint_as_float(w0 << 8);
+  f[1] = __uint_as_float(__byte_perm(w0, w1, 0x5430) & 0xFFFFFF00u);
+  f[2] = __uint_as_float(__byte_perm(w1, w2, 0x4320) & 0xFFFFFF00u);
+  f[3] = __uint_as_float(w2 & 0xFFFFFF00u);
 }
 
 MLA_DEV uint32_t pack_bf16x2(float lo, float hi) {

@@ -11,3 +11,14 @@ if ROOT not in sys.path:
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a B200 (sm_100a) GPU")
     config.addinivalue_line("markers", "slow: takes more than a few seconds on CPU")
+
+
+@pytest.fixture(scope="session")
+def libmla():
+    """Builds libmla.so in-tree if needed and returns the binding module."""
+    from mla_latent_kv_26_b200 import build
+
+    build.build()
+    from mla_latent_kv_26_b200 import binding
+
+    return binding

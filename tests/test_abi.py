@@ -1,0 +1,112 @@
+"""CPU-side checks of the C ABI: the library loads, exports every function
+include/mla.h declares, and rejects bad arguments before touching a GPU."""
+
+import ctypes
+import math
+import os
+import re
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    names = []
+    for f in os.listdir(os.path.join(ROOT, "include")):
+        if f.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", f)).read()
+            names += re.findall(r"MLA_API\s+[\w\s\*]+?\b(mla_\w+)\s*\(", text)
+    return sorted(set(names))
+
+
+def test_header_declares_the_boundary():
+    assert _declared() == sorted([
+        "mla_combine", "mla_decode", "mla_decode_plan", "mla_get_error", "mla_num_workers", "mla_plan_bytes",
+        "mla_status_string", "mla_workspace_bytes"])
+
+
+def test_library_exports_every_declared_symbol(libmla):
+    lib = ctypes.CDLL(libmla.LIB_PATH)
+    for name in _declared():
+        assert hasattr(lib, name), name
+    assert set(_declared()) == set(libmla.EXPORTED)
+    out = subprocess.run(["nm", "-D", "--defined-only", libmla.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r" T (mla_\w+)", out))
+    assert exported == set(_declared())
+
+
+def _desc(libmla, **kw):
+    base = dict(batch=2, q_len=1, num_heads=128, num_pages=8, max_pages_per_seq=4)
+    base.update(kw)
+    return libmla.make_desc(**base)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(batch=-1), 1), (dict(q_len=0), 1), (dict(num_pages=0), 1), (dict(max_pages_per_seq=0), 1),
+    (dict(topk=-3), 1), (dict(causal=True, topk=4), 1), (dict(softmax_scale=0.0), 1),
+    (dict(softmax_scale=float("nan")), 1), (dict(softmax_scale=float("inf")), 1),
+    (dict(d_latent=256), 2), (dict(d_rope=32), 2), (dict(page_size=16), 2), (dict(num_heads=24), 2),
+    (dict(num_heads=256), 2), (dict(num_heads=8), 2),
+])
+def test_bad_descriptors_rejected_before_launch(libmla, kw, status):
+    d = _desc(libmla, **kw)
+    assert libmla.mla_plan_bytes(d) == 0
+    assert libmla.mla_workspace_bytes(d) == 0
+    assert libmla.mla_num_workers(d) == 0
+    assert libmla.mla_decode_plan(d, 16, 16, 1 << 20, None) == status
+    assert libmla.mla_decode(d, 16, 16, 16, 16, 16, 16, 16, 16, 16, 1 << 30, None) == status
+    assert libmla.mla_combine(d, 16, 16, 1 << 30, 16, 16, None) == status
+
+
+def test_null_and_misaligned_pointers_rejected(libmla):
+    d = _desc(libmla)
+    INV = libmla.MLA_ERR_INVALID_ARG
+    assert libmla.mla_decode_plan(d, None, 16, 1 << 20, None) == INV
+    assert libmla.mla_decode_plan(d, 16, None, 1 << 20, None) == INV
+    assert libmla.mla_decode_plan(d, 16, 8, 1 << 20, None) == INV            # plan not 16-B aligned
+    args = [16] * 9
+    for i in range(9):
+        a = list(args)
+        a[i] = None
+        if i == 5:      # topk_indices may be NULL for a dense descriptor: that alone is not an error
+            continue
+        assert libmla.mla_decode(d, *a[:9], 1 << 30, None) == INV, i
+    # misaligned q / cache / out
+    for i in (1, 2, 6):
+        a = list(args)
+        a[i] = 24
+        assert libmla.mla_decode(d, *a, 1 << 30, None) == INV, i
+    sparse = _desc(libmla, topk=8)
+    a = list(args)
+    a[5] = None
+    assert libmla.mla_decode(sparse, *a, 1 << 30, None) == INV
+    assert libmla.mla_combine(d, None, 16, 1 << 30, 16, 16, None) == INV
+    assert libmla.mla_combine(d, 16, 16, 1 << 30, 16, 18, None) == INV       # lse not 4-B aligned
+    st, _ = libmla.mla_get_error(None)
+    assert st == INV
+
+
+def test_plan_too_small_rejected(libmla):
+    d = _desc(libmla)
+    need = libmla.mla_plan_bytes(d)
+    assert need == ((8 + 2 * 2 + 1) * 4 + 15) // 16 * 16
+    assert libmla.mla_decode_plan(d, 16, 16, need - 4, None) == libmla.MLA_ERR_WORKSPACE_TOO_SMALL
+
+
+def test_status_strings(libmla):
+    seen = set()
+    for s in range(7):
+        txt = libmla.mla_status_string(s)
+        assert txt and txt not in seen
+        seen.add(txt)
+    assert libmla.mla_status_string(99) == "unknown status"
+
+
+def test_binding_fails_loudly_without_library():
+    env = dict(os.environ, MLA_LIB="/nonexistent/libmla.so")
+    code = "import mla_latent_kv_26_b200.binding"
+    r = subprocess.run([sys.executable, "-c", code], cwd=ROOT, env=env, capture_output=True, text=True)
+    assert r.returncode != 0 and "libmla.so is not built" in r.stderr
