@@ -165,6 +165,7 @@ mla_status_t mla_decode(const mla_decode_desc_t* desc, void* plan, const void* q
                         float* lse, void* workspace, size_t workspace_bytes, mla_stream_t stream) {
   mla_status_t st = check_desc(desc);
   if (st != MLA_OK) return st;
+  if (desc->batch == 0) return MLA_OK;  // nothing to read or write; empty tensors may be NULL
   if (!plan || !q || !kv_cache || !block_table || !seq_lens || !out || !lse || !workspace)
     return MLA_ERR_INVALID_ARG;
   if (desc->topk > 0 && !topk_indices) return MLA_ERR_INVALID_ARG;
@@ -176,7 +177,6 @@ mla_status_t mla_decode(const mla_decode_desc_t* desc, void* plan, const void* q
   if (!device_info(&info)) return MLA_ERR_CUDA;
   const int workers = workers_for(desc, info);
   if (workspace_bytes < workspace_bytes_for(desc, workers)) return MLA_ERR_WORKSPACE_TOO_SMALL;
-  if (desc->batch == 0) return MLA_OK;
 
   PFN_cuTensorMapEncodeTiled_v12000 enc = encoder();
   if (!enc) return MLA_ERR_CUDA;
@@ -221,6 +221,7 @@ mla_status_t mla_combine(const mla_decode_desc_t* desc, void* plan, const void* 
                          void* out, float* lse, mla_stream_t stream) {
   mla_status_t st = check_desc(desc);
   if (st != MLA_OK) return st;
+  if (desc->batch == 0) return MLA_OK;
   if (!plan || !workspace || !out || !lse) return MLA_ERR_INVALID_ARG;
   if (!aligned16(plan) || !aligned16(workspace) || !aligned16(out) || ((uintptr_t)lse & 3u))
     return MLA_ERR_INVALID_ARG;
