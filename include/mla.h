@@ -139,6 +139,33 @@ MLA_API mla_status_t mla_combine(const mla_decode_desc_t* desc, void* plan, cons
  * (timeout bit set) or MLA_ERR_DEVICE_BOUNDS (any other bit). */
 MLA_API mla_status_t mla_get_error(const void* plan, uint32_t* error_bits, mla_stream_t stream);
 
+/* Decode step with no device allocation by anyone: plan + decode + combine as
+ * above, with the plan and the split partials kept in a fixed 32 MiB array of
+ * device memory that the library itself defines (every device that loads
+ * libmla holds it until the process exits). For callers that cannot call
+ * cudaMalloc, for example code running where a caching allocator owns all
+ * device memory, or an embedding that forbids allocation while serving.
+ * The caller passes inputs and outputs as for mla_decode_plan / mla_decode.
+ * The paper has no counterpart; this is an interface convenience.
+ *
+ * - The first call on a device sets up the scratch's device address and the
+ *   kernel attributes (with that device current); make that first call before
+ *   any stream capture.
+ * - The plan and the partials are rewritten by every call before they are
+ *   read, so nothing has to start at zero; the array keeps the last call's
+ *   contents. All calls share it: calls that overlap on the GPU (other
+ *   streams, other threads) race and give wrong results. Serialise them.
+ * - If the plan plus the worst-case partials (one per worker and task, at
+ *   H x 2 KiB each) do not fit, fewer workers are used; if even one worker
+ *   does not fit (roughly more than 120 query tokens of 128 heads per call),
+ *   returns MLA_ERR_WORKSPACE_TOO_SMALL before any launch.
+ * - Device-side errors are handled as in mla_decode (bad tokens skipped) but
+ *   the error word is not reachable by the caller; use the allocating entry
+ *   points to read it. */
+MLA_API mla_status_t mla_decode_noalloc(const mla_decode_desc_t* desc, const int32_t* seq_lens, const void* q,
+                                        const void* kv_cache, const int32_t* block_table,
+                                        const int32_t* topk_indices, void* out, float* lse, mla_stream_t stream);
+
 /* Static string for a status code. */
 MLA_API const char* mla_status_string(mla_status_t status);
 

@@ -29,7 +29,7 @@ MLA_DEVERR_TIMEOUT = 0x8
 
 EXPORTED = (
     "mla_plan_bytes", "mla_workspace_bytes", "mla_num_workers", "mla_decode_plan", "mla_decode",
-    "mla_combine", "mla_get_error", "mla_status_string",
+    "mla_combine", "mla_get_error", "mla_status_string", "mla_decode_noalloc",
 )
 
 DEFAULT_SOFTMAX_SCALE = 1.0 / math.sqrt(192.0)
@@ -76,6 +76,7 @@ def _load() -> ctypes.CDLL:
         "mla_combine": (ctypes.c_int, [D, P, P, ctypes.c_size_t, P, P, P]),
         "mla_get_error": (ctypes.c_int, [P, ctypes.POINTER(ctypes.c_uint32), P]),
         "mla_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+        "mla_decode_noalloc": (ctypes.c_int, [D, P, P, P, P, P, P, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -140,6 +141,12 @@ def mla_decode(desc, plan, q, kv_cache, block_table, seq_lens, topk_indices, out
 def mla_combine(desc, plan, workspace, workspace_bytes: int, out, lse, stream=None) -> int:
     return int(_lib.mla_combine(ctypes.byref(desc), _ptr(plan), _ptr(workspace), int(workspace_bytes), _ptr(out),
                                 _ptr(lse), _stream(stream)))
+
+
+def mla_decode_noalloc(desc, seq_lens, q, kv_cache, block_table, topk_indices, out, lse, stream=None) -> int:
+    """Plan + decode + combine with the library's fixed device scratch (no allocation)."""
+    return int(_lib.mla_decode_noalloc(ctypes.byref(desc), _ptr(seq_lens), _ptr(q), _ptr(kv_cache), _ptr(block_table),
+                                       _ptr(topk_indices), _ptr(out), _ptr(lse), _stream(stream)))
 
 
 def mla_get_error(plan, stream=None):

@@ -269,3 +269,81 @@ const char* mla_status_string(mla_status_t s) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// mla_decode_noalloc: the full decode step (plan + decode + combine) with its
+// scratch (plan buffer and split partials) in a fixed array of device memory
+// that this library defines, for callers that cannot allocate device memory.
+
+namespace mla {
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = 32u << 20;  // 32 MiB, held by every device that loads the library
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of the scratch array for the current device. In host code
+// the array's name is only a stand-in, so the address is looked up once per
+// device (the first call on a device does it, with that device current).
+bool noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
+      cudaGetLastError();
+      return false;
+    }
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return true;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+}  // namespace
+}  // namespace mla
+
+extern "C" mla_status_t mla_decode_noalloc(const mla_decode_desc_t* desc, const int32_t* seq_lens, const void* q,
+                                           const void* kv_cache, const int32_t* block_table,
+                                           const int32_t* topk_indices, void* out, float* lse,
+                                           mla_stream_t stream) {
+  mla_status_t st = check_desc(desc);
+  if (st != MLA_OK) return st;
+  if (desc->batch == 0) return MLA_OK;
+  if (!seq_lens || !q || !kv_cache || !block_table || !out || !lse) return MLA_ERR_INVALID_ARG;
+  if (desc->topk > 0 && !topk_indices) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(kv_cache) || !aligned16(out) || ((uintptr_t)lse & 3u) ||
+      ((uintptr_t)block_table & 3u) || ((uintptr_t)seq_lens & 3u) || ((uintptr_t)topk_indices & 3u))
+    return MLA_ERR_INVALID_ARG;  // checked here so that nothing is launched for a bad call
+  DeviceInfo info;
+  if (!device_info(&info)) return MLA_ERR_CUDA;
+  void* scratch = nullptr;
+  if (!noalloc_scratch(&scratch)) return MLA_ERR_CUDA;
+
+  // Scratch layout: [plan | partial outputs | partial LSEs]. The split
+  // partials need one slot per (worker, task) overlap, worst case
+  // workers + tasks; use fewer workers when that does not fit.
+  const size_t plan_bytes = plan_bytes_for(desc);
+  const size_t per_slot = part_o_bytes(1, desc->num_heads) + part_lse_bytes(1, desc->num_heads);
+  const long long tasks = (long long)desc->batch * desc->q_len;
+  const long long max_slots = (long long)((kNoAllocScratchBytes - align256(plan_bytes)) / per_slot);
+  long long workers = workers_for(desc, info);
+  if (workers + tasks > max_slots) workers = max_slots - tasks;
+  if (workers < 1) return MLA_ERR_WORKSPACE_TOO_SMALL;  // batch too large for the fixed scratch
+
+  mla_decode_desc_t d = *desc;
+  d.num_sms = (int32_t)(2 * workers);
+  void* plan = scratch;
+  void* ws = static_cast<char*>(scratch) + align256(plan_bytes);
+  const size_t ws_bytes = workspace_bytes_for(&d, (int)workers);
+  st = mla_decode_plan(&d, seq_lens, plan, plan_bytes, stream);
+  if (st != MLA_OK) return st;
+  st = mla_decode(&d, plan, q, kv_cache, block_table, seq_lens, topk_indices, out, lse, ws, ws_bytes, stream);
+  if (st != MLA_OK) return st;
+  return mla_combine(&d, plan, ws, ws_bytes, out, lse, stream);
+}

@@ -24,8 +24,8 @@ def _declared():
 
 def test_header_declares_the_boundary():
     assert _declared() == sorted([
-        "mla_combine", "mla_decode", "mla_decode_plan", "mla_get_error", "mla_num_workers", "mla_plan_bytes",
-        "mla_status_string", "mla_workspace_bytes"])
+        "mla_combine", "mla_decode", "mla_decode_noalloc", "mla_decode_plan", "mla_get_error", "mla_num_workers",
+        "mla_plan_bytes", "mla_status_string", "mla_workspace_bytes"])
 
 
 def test_library_exports_every_declared_symbol(libmla):
