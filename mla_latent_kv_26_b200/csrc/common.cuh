@@ -1,6 +1,7 @@
 // Definitions shared by the libmla kernels and the host entry points.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <stdint.h>
 
@@ -45,6 +46,17 @@ struct DecodeArgs {
   int32_t* plan;
   int batch, q_len, heads, num_pages, max_pages_per_seq, topk;
   float scale_log2;             // softmax_scale * log2(e)
+};
+
+// Tensor maps of the cache viewed as a 2-D tensor [num_pages * 64 rows, 576
+// columns] of bf16: boxes of 64 columns (128-byte swizzle) and of 32 columns
+// (64-byte swizzle), each 64 rows high for page tiles and 1 row high for
+// gathers.
+struct CacheMaps {
+  CUtensorMap tile;
+  CUtensorMap row;
+  CUtensorMap rope_tile;
+  CUtensorMap rope_row;
 };
 
 struct CombineArgs {

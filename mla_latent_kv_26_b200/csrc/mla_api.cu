@@ -16,7 +16,7 @@ cudaError_t launch_combine(const CombineArgs& args, int tasks, cudaStream_t stre
 const void* decode_kernel_ptr();
 int decode_smem_bytes();
 int decode_threads();
-cudaError_t launch_decode(const CUtensorMap& tm_tile, const CUtensorMap& tm_row, const DecodeArgs& args, int workers,
+cudaError_t launch_decode(const CacheMaps& maps, const DecodeArgs& args, int workers,
                           cudaStream_t stream);
 
 namespace {
@@ -180,20 +180,22 @@ mla_status_t mla_decode(const mla_decode_desc_t* desc, void* plan, const void* q
 
   PFN_cuTensorMapEncodeTiled_v12000 enc = encoder();
   if (!enc) return MLA_ERR_CUDA;
-  // The cache as a 2-D tensor [num_pages * 64 rows, 576 columns] of bf16.
-  CUtensorMap tm_tile, tm_row;
+  // The cache as a 2-D tensor [num_pages * 64 rows, 576 columns] of bf16:
+  // 64-column boxes with 128-byte swizzle (latent columns) and 32-column
+  // boxes with 64-byte swizzle (rope columns), 64 rows (page) or 1 row (gather).
+  CacheMaps maps;
   cuuint64_t dims[2] = {(cuuint64_t)kDQK, (cuuint64_t)desc->num_pages * kPage};
   cuuint64_t strides[1] = {(cuuint64_t)kDQK * 2};
-  cuuint32_t box_tile[2] = {64, 64};
-  cuuint32_t box_row[2] = {64, 1};
   cuuint32_t elem[2] = {1, 1};
-  if (enc(&tm_tile, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(kv_cache), dims, strides, box_tile, elem,
-          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-    return MLA_ERR_CUDA;
-  if (enc(&tm_row, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(kv_cache), dims, strides, box_row, elem,
-          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+  auto encode = [&](CUtensorMap* m, cuuint32_t cols, cuuint32_t rows, CUtensorMapSwizzle sw) {
+    cuuint32_t box[2] = {cols, rows};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(kv_cache), dims, strides, box, elem,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  };
+  if (!encode(&maps.tile, 64, kPage, CU_TENSOR_MAP_SWIZZLE_128B) || !encode(&maps.row, 64, 1, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode(&maps.rope_tile, 32, kPage, CU_TENSOR_MAP_SWIZZLE_64B) ||
+      !encode(&maps.rope_row, 32, 1, CU_TENSOR_MAP_SWIZZLE_64B))
     return MLA_ERR_CUDA;
 
   const int slots = workers + desc->batch * desc->q_len;
@@ -214,7 +216,7 @@ mla_status_t mla_decode(const mla_decode_desc_t* desc, void* plan, const void* q
   a.max_pages_per_seq = desc->max_pages_per_seq;
   a.topk = desc->topk;
   a.scale_log2 = desc->softmax_scale * 1.4426950408889634f;
-  return launch_decode(tm_tile, tm_row, a, workers, (cudaStream_t)stream) == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+  return launch_decode(maps, a, workers, (cudaStream_t)stream) == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
 mla_status_t mla_combine(const mla_decode_desc_t* desc, void* plan, const void* workspace, size_t workspace_bytes,

@@ -1,49 +1,50 @@
 // Steps a2-a7: split-KV MLA decode over the paged latent cache on sm_100a.
 //
 // One worker = a cluster of two CTAs on two SMs. A task (one query token of
-// one sequence, up to 128 heads) is processed by both CTAs together:
-//
-//   CTA rank 0: loads cache columns [0, 320); partial scores over columns
-//               [0, 288); output columns [0, 256)
-//   CTA rank 1: loads cache columns [256, 576); partial scores over [288, 576);
-//               output columns [256, 512)
+// one sequence, up to 128 heads) is processed by both CTAs together; CTA rank
+// r loads, for every 64-token tile, cache columns [256r, 256r + 256) (its
+// output columns) and [512 + 32r, 512 + 32r + 32) (half of the rope part),
+// and contracts its partial scores over those 288 columns.
 //
 // The fp32 output accumulator of 128 heads x 512 columns is exactly one SM's
 // tensor memory, so the pair splits the output columns, and the score
 // contraction with them. The softmax of each head row is owned by one CTA:
 // in every 32-lane TMEM quadrant, CTA r owns lanes [16r, 16r+16). For each
-// 64-token tile, a CTA sends the peer the partial scores of the rows the peer
-// owns (24-bit floats, fp32 rounded to its top three bytes, relative error
-// <= 2^-16; 12 KB), receives the peer's partials of its own rows, runs the
-// online softmax for its 64 rows, and sends back their P (bf16) together with
-// the per-row rescale factor, running max and running sum (9 KB). Both CTAs
-// then hold the same P for all 128 rows and accumulate their output halves
-// with it. (The SM-to-SM path sustains ~15 B/clk per direction, so the
-// exchange volume, not the arithmetic, decides this layout.)
+// tile, a CTA sends the peer the partial scores of the rows the peer owns
+// (16-bit block fixed point, one power-of-two scale per row; 8 KB),
+// receives the peer's partials of its own rows, runs the online softmax for
+// its 64 rows, and sends back their P (bf16) together with the per-row
+// rescale factor, running max and running sum (9 KB). Both CTAs then hold the
+// same P for all 128 rows and accumulate their output halves with it.
 //
-// Per CTA (320 threads):
+// Per CTA (448 threads):
 //   warp 0      TMA producer: 64-token pages (block table) or 64 gathered rows
-//               (top-k indices, tile::gather4) into a 4-stage ring, 5 boxes of
-//               64 rows x 128 B (128-byte swizzle) per stage
+//               (top-k indices, tile::gather4) into a 4-stage ring; a stage is
+//               four boxes of 64 rows x 128 B (128-byte swizzle) and one box
+//               of 64 rows x 64 B (64-byte swizzle)
 //   warp 1      tcgen05 issuer: S = Q_slice * K_slice^T (M=128 heads, N=64
-//               tokens, K=288, A = Q in TMEM) one tile ahead of
-//               O += P * V (M=128, N=256, K=64, A = P in shared memory, B = the
-//               same stage read MN-major); it polls both queues and issues
-//               whichever is ready
+//               tokens, K=288; A = Q in TMEM, its rope columns from shared
+//               memory) into one of two S buffers, and O += P * V (M=128,
+//               N=256, K=64, A = P in shared memory, B = the stage read
+//               MN-major); it polls both queues, PV first
 //   warps 2-5   softmax, one per quadrant: 16 owned rows x 64 tokens, two
 //               threads per row (16x32bx2 TMEM accesses); P of the owned rows
 //               into this CTA's P buffer and, by one bulk copy per quadrant,
 //               into the peer's; epilogue of the owned rows
-//   warps 6-9   helpers, one per quadrant, for the rows the peer owns: send
-//               their partial scores, apply the peer's rescale factors, epilogue
-//               of those rows; warp 8 also relays "receive slot read" tokens
+//   warps 6-9   senders, one per quadrant, for the rows the peer owns: send
+//               their partial scores; warp 8 also relays "receive slot read"
+//               tokens
+//   warps 10-13 acceptors, one per quadrant, for the rows the peer owns: apply
+//               the peer's rescale factors, epilogue of those rows
 //
-// P is double-buffered in shared memory (128 heads x 64 tokens bf16, K-major,
-// 128-byte swizzle, identical offsets in both CTAs). The PV commit arrives on
-// the P-buffer barrier of both CTAs, so a buffer is rewritten only after both
-// CTAs' PV of two tiles earlier completed.
+// S is double-buffered in TMEM, so the S of tile k + 1 (and its exchange)
+// proceeds while the softmax warps work on tile k. P is double-buffered in
+// shared memory (128 heads x 64 tokens bf16, K-major, 128-byte swizzle,
+// identical offsets in both CTAs). The PV commit arrives on the P-buffer
+// barrier of both CTAs, so a buffer is rewritten only after both CTAs' PV of
+// two tiles earlier completed.
 //
-// TMEM columns: O [0,256) | Q [256,400) | S [400,464).
+// TMEM columns: O [0,256) | Q [256,384) | S buffers [384,448), [448,512).
 #include <cuda.h>
 #include <math.h>
 
@@ -55,41 +56,51 @@ namespace dec {
 
 using namespace ptx;
 
-constexpr int kThreads = 320;
+constexpr int kThreads = 448;
 constexpr int kStages = 4;
 constexpr int kBoxBytes = kPage * 128;  // 64 rows x 64 bf16 (one 128-B swizzle row each)
-constexpr int kBoxesPerStage = 5;       // 320 columns per CTA
-constexpr int kStageBytes = kBoxesPerStage * kBoxBytes;
-constexpr int kSSteps = 18;             // 288 columns / 16 per MMA
+constexpr int kVBoxes = 4;              // this CTA's 256 output columns, 4 boxes of 64
+constexpr int kRopeBoxBytes = kPage * 64;  // 64 rows x 32 bf16 (one 64-byte swizzle row each)
+constexpr int kRopeOff = kVBoxes * kBoxBytes;
+constexpr int kStageBytes = kRopeOff + kRopeBoxBytes;
 // Partial-score slot: per quadrant, 32 threads x 6 chunks of 16 B (16 rows x 64 tokens x 3 B).
-constexpr int kXQuadBytes = 32 * 6 * 16;
-constexpr int kXBytes = 4 * kXQuadBytes;
+// Score slot: per quadrant, 32 threads x 4 chunks of 16 B (16 rows x 64
+// tokens of 16-bit fixed point), then per quadrant 16 row exponents of 4 B.
+constexpr int kXQuadBytes = 32 * 4 * 16;
+constexpr int kXExpBytes = 16 * 4;
+constexpr int kXExpOff = 4 * kXQuadBytes;
+constexpr int kXBytes = kXExpOff + 4 * kXExpBytes;
 // P buffer: 128 rows of 64 bf16 (one 128-byte swizzle row each).
 constexpr int kPSlotBytes = 128 * 128;
 constexpr int kPQuadBytes = 16 * 128;    // the 16 rows a CTA owns in one quadrant
 // Rescale factor, running max and running sum of the peer's rows: 16 B per row.
 constexpr int kStatBytes = 64 * 16;
 constexpr int kStatQuadBytes = 16 * 16;
-constexpr int kXSlots = 2;
+constexpr int kPSlots = 2;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kTmemO = 0, kTmemQ = 256, kTmemS = 400;
+// Q: this CTA's 256 output columns in TMEM (two bf16 per TMEM column), its
+// 32 rope columns in shared memory (no-swizzle K-major core matrices of 8
+// rows x 16 B). S buffer b (tile k uses b = k % 2) starts at kTmemS + 64 b.
+constexpr uint32_t kTmemO = 0, kTmemQ = 256, kTmemS = 384;
+constexpr int kQRopeBytes = 128 * 64;  // 128 rows x 32 bf16
+constexpr uint32_t kQRopeLbo = 128, kQRopeSbo = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: tolerate p up to 2^8 before rescaling O
 constexpr uint64_t kTimeoutNs = 2000000000ull;
-// Shared memory: [misc | stage ring | P buffers | score slots | stat slots];
+// Shared memory: [misc | stage ring | P buffers | score slot | stat slots | Q rope];
 // the stage ring and the P buffers must be 1024-byte aligned (128-byte
 // swizzle atoms), which holds when the dynamic shared memory base is (checked
 // at run time).
-constexpr int kMiscBytes = 3072;
-constexpr int kSmemBytes = kMiscBytes + kStages * kStageBytes + kXSlots * (kPSlotBytes + kXBytes + kStatBytes);
+constexpr int kMiscBytes = 1024;
+constexpr int kSmemBytes =
+    kMiscBytes + kStages * kStageBytes + kPSlots * (kPSlotBytes + kStatBytes) + kXBytes + kQRopeBytes;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 
 struct Misc {
   uint64_t full[kStages];
   uint64_t empty[kStages];
-  uint64_t s_full, s_free, o_full, o_empty, q_full, mma_done;
-  uint64_t p_full[kXSlots], p_free[kXSlots];
-  uint64_t x_full[kXSlots], x_empty[kXSlots], x_read[kXSlots];
-  uint64_t pm_full[kXSlots];
+  uint64_t s_full[2], s_free[2], o_full, o_empty, q_full, mma_done;
+  uint64_t p_full[kPSlots], p_free[kPSlots], pm_full[kPSlots];
+  uint64_t x_full, x_empty, x_read;
   uint64_t stage_mask[kStages];
   uint32_t tmem_base;
   uint32_t abort_flag;
@@ -175,15 +186,15 @@ struct Cursor {
 };
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
-    mla_decode_kernel(const __grid_constant__ CUtensorMap tm_tile, const __grid_constant__ CUtensorMap tm_row,
-                      const DecodeArgs a) {
+    mla_decode_kernel(const __grid_constant__ CacheMaps maps, const DecodeArgs a) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   Misc* misc = reinterpret_cast<Misc*>(smem_raw);
   const uint32_t raw_base = smem_addr(smem_raw);
   const uint32_t stage_base = raw_base + kMiscBytes;
   const uint32_t pbuf = stage_base + kStages * kStageBytes;  // P buffers (1024-aligned)
-  const uint32_t xbuf = pbuf + kXSlots * kPSlotBytes;         // score slots
-  const uint32_t statbuf = xbuf + kXSlots * kXBytes;          // stat slots
+  const uint32_t xbuf = pbuf + kPSlots * kPSlotBytes;         // score slot
+  const uint32_t statbuf = xbuf + kXBytes;                    // stat slots
+  const uint32_t qrope = statbuf + kPSlots * kStatBytes;      // rope columns of Q
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t crank = cluster_ctarank();
@@ -200,26 +211,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       mbar_init(smem_addr(&misc->full[s]), 1);
       mbar_init(smem_addr(&misc->empty[s]), 1);
     }
-    mbar_init(smem_addr(&misc->s_full), 1);
-    mbar_init(smem_addr(&misc->s_free), 8);   // 4 softmax + 4 helper warps
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(smem_addr(&misc->s_full[b]), 1);
+      mbar_init(smem_addr(&misc->s_free[b]), 8);   // 4 softmax + 4 sender warps
+    }
     mbar_init(smem_addr(&misc->o_full), 1);
-    mbar_init(smem_addr(&misc->o_empty), 8);
-    mbar_init(smem_addr(&misc->q_full), 8);
+    mbar_init(smem_addr(&misc->o_empty), 8);  // 4 softmax + 4 acceptor warps
+    mbar_init(smem_addr(&misc->q_full), 8);   // 4 softmax + 4 sender warps
     mbar_init(smem_addr(&misc->mma_done), 1);
-    for (int xs = 0; xs < kXSlots; ++xs) {
-      mbar_init(smem_addr(&misc->x_full[xs]), 1);
-      mbar_init(smem_addr(&misc->x_empty[xs]), 1);
-      mbar_init(smem_addr(&misc->x_read[xs]), 4);
-      mbar_init(smem_addr(&misc->pm_full[xs]), 1);
-      mbar_init(smem_addr(&misc->p_full[xs]), 8);   // 4 softmax + 4 helper warps
-      mbar_init(smem_addr(&misc->p_free[xs]), 2);   // the PV commits of both CTAs
+    mbar_init(smem_addr(&misc->x_full), 1);
+    mbar_init(smem_addr(&misc->x_empty), 1);
+    mbar_init(smem_addr(&misc->x_read), 4);
+    for (int ps = 0; ps < kPSlots; ++ps) {
+      mbar_init(smem_addr(&misc->pm_full[ps]), 1);
+      mbar_init(smem_addr(&misc->p_full[ps]), 8);   // 4 softmax + 4 acceptor warps
+      mbar_init(smem_addr(&misc->p_free[ps]), 2);   // the PV commits of both CTAs
     }
     misc->abort_flag = 0u;
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
-    prefetch_tmap(&tm_tile);
-    prefetch_tmap(&tm_row);
+    prefetch_tmap(&maps.tile);
+    prefetch_tmap(&maps.row);
+    prefetch_tmap(&maps.rope_tile);
+    prefetch_tmap(&maps.rope_row);
   }
   if (warp == 1) {
     tmem_alloc(smem_addr(&misc->tmem_base), kTmemCols);
@@ -229,7 +244,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   cluster_sync();
   tc_fence_after();
   const uint32_t tmem = misc->tmem_base;
-  const int col0 = crank ? 256 : 0;  // first cache column loaded by this CTA
+  // Cache columns of this CTA: output columns [vcol0, vcol0 + 256) in four
+  // 128-byte-swizzled boxes, and rope columns [rcol0, rcol0 + 32) in one
+  // 64-byte-swizzled box; the scores are contracted over both (288 columns).
+  const int vcol0 = 256 * (int)crank;
+  const int rcol0 = kDLatent + 32 * (int)crank;
 
   Cursor cur;
   cur.init(a.plan, worker);
@@ -238,7 +257,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   int task = 0, pg0 = 0, pg1 = 0;
   bool split = false;
 
-  // Quadrant roles shared by the softmax and helper warps.
+  // Quadrant roles shared by the softmax, sender and acceptor warps.
   const int quad = warp & 3;
   const bool quad_active = quad * 32 < a.heads;
   const uint32_t n_active = (uint32_t)((a.heads + 31) / 32);
@@ -249,30 +268,45 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const uint32_t own_lanes = tmem + ((uint32_t)(quad * 32 + 16 * (int)crank) << 16);
   const uint32_t peer_lanes = tmem + ((uint32_t)(quad * 32 + 16 * (int)peer) << 16);
 
-  // Q (this CTA's 288 columns) into TMEM: the softmax warp writes columns
-  // [0,144) of its quadrant's 32 rows, the helper warp [144,288).
+  // Q (this CTA's 288 score columns): the softmax warp writes
+  // Q[vcol0, vcol0 + 128) of its quadrant's 32 rows into TMEM, the sender
+  // warp Q[vcol0 + 128, vcol0 + 256) into TMEM and Q[rcol0, rcol0 + 32) into
+  // shared memory.
   auto write_q = [&](int half) {
     const int row = quad * 32 + lane;
     const size_t qrow = (size_t)task * a.heads + row;
-    uint32_t qv[72];
-    if (row < a.heads) {
-      const uint4* src = reinterpret_cast<const uint4*>(a.q + qrow * kDQK + crank * 288 + half * 144);
+    const bool valid = row < a.heads;
+    const uint4* src = reinterpret_cast<const uint4*>(a.q + qrow * kDQK + vcol0 + half * 128);
+    uint32_t qv[64];
 #pragma unroll
-      for (int u = 0; u < 18; ++u) {
-        const uint4 v = src[u];
-        qv[4 * u + 0] = v.x;
-        qv[4 * u + 1] = v.y;
-        qv[4 * u + 2] = v.z;
-        qv[4 * u + 3] = v.w;
-      }
-    } else {
-#pragma unroll
-      for (int u = 0; u < 72; ++u) qv[u] = 0u;
+    for (int u = 0; u < 16; ++u) {
+      const uint4 v = valid ? src[u] : make_uint4(0, 0, 0, 0);
+      qv[4 * u + 0] = v.x;
+      qv[4 * u + 1] = v.y;
+      qv[4 * u + 2] = v.z;
+      qv[4 * u + 3] = v.w;
     }
-    const uint32_t qa = tmem + ((uint32_t)(quad * 32) << 16) + kTmemQ + 72 * half;
+    const uint32_t qa = tmem + ((uint32_t)(quad * 32) << 16) + kTmemQ + 64 * half;
     tmem_st_32(qa, *reinterpret_cast<const uint32_t(*)[32]>(&qv[0]));
     tmem_st_32(qa + 32, *reinterpret_cast<const uint32_t(*)[32]>(&qv[32]));
-    tmem_st_8(qa + 64, *reinterpret_cast<const uint32_t(*)[8]>(&qv[64]));
+    if (half == 1) {
+      const uint4* rsrc = reinterpret_cast<const uint4*>(a.q + qrow * kDQK + rcol0);
+      uint32_t rv[16];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const uint4 v = valid ? rsrc[u] : make_uint4(0, 0, 0, 0);
+        rv[4 * u + 0] = v.x;
+        rv[4 * u + 1] = v.y;
+        rv[4 * u + 2] = v.z;
+        rv[4 * u + 3] = v.w;
+      }
+      // core matrix (row / 8, column / 8) of 8 rows x 16 B
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        st_shared_v4(qrope + (uint32_t)(row >> 3) * kQRopeSbo + (uint32_t)u * kQRopeLbo + (uint32_t)(row & 7) * 16u,
+                     make_uint4(rv[4 * u], rv[4 * u + 1], rv[4 * u + 2], rv[4 * u + 3]));
+      fence_proxy_async_smem();  // read by the tensor core
+    }
     tmem_wait_st();
     tc_fence_before();
     __syncwarp();
@@ -327,14 +361,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       else if (write_lse) a.lse[qrow] = lse;
     }
   };
-  // Drain the last phases of a slot barrier fed by 4-byte remote tokens.
-  auto drain_tokens = [&](uint64_t* bars, int uses_total, uint32_t bytes, bool expect) {
-    for (int xs = 0; xs < kXSlots; ++xs) {
-      const int uses = (uses_total + 1 - xs) / 2;
-      if (uses > 0) {
-        if (expect) mbar_arrive_expect_tx(smem_addr(&bars[xs]), bytes);
-        W.wait_cluster_warp(&bars[xs], (uses - 1) & 1);
-      }
+  // The last phase of the score-slot barrier, fed by the peer's 4-byte "slot
+  // read" token for every tile sent, is collected before exit.
+  auto drain_x_empty = [&](int tiles, bool expect) {
+    if (tiles > 0) {
+      if (expect) mbar_arrive_expect_tx(smem_addr(&misc->x_empty), 4u);
+      W.wait_cluster_warp(&misc->x_empty, (tiles - 1) & 1);
     }
   };
 
@@ -371,8 +403,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
               const int row = (ok ? page : 0) * kPage;
               const uint32_t dst = stage_base + s * kStageBytes;
 #pragma unroll
-              for (int bx = 0; bx < kBoxesPerStage; ++bx)
-                tma_load_2d(dst + bx * kBoxBytes, &tm_tile, col0 + 64 * bx, row, fb);
+              for (int bx = 0; bx < kVBoxes; ++bx)
+                tma_load_2d(dst + bx * kBoxBytes, &maps.tile, vcol0 + 64 * bx, row, fb);
+              tma_load_2d(dst + kRopeOff, &maps.rope_tile, rcol0, row, fb);
             }
             __syncwarp();
           }
@@ -418,10 +451,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           }
           __syncwarp();
           if (lane < 16) {
-            const uint32_t dst = stage_base + s * kStageBytes + lane * 4 * 128;
+            // lane l gathers tile rows 4l .. 4l+3
+            const uint32_t dst = stage_base + s * kStageBytes;
 #pragma unroll
-            for (int bx = 0; bx < kBoxesPerStage; ++bx)
-              tma_gather4(dst + bx * kBoxBytes, &tm_row, col0 + 64 * bx, r[0], r[1], r[2], r[3], fb);
+            for (int bx = 0; bx < kVBoxes; ++bx)
+              tma_gather4(dst + bx * kBoxBytes + lane * 4 * 128, &maps.row, vcol0 + 64 * bx, r[0], r[1], r[2], r[3], fb);
+            tma_gather4(dst + kRopeOff + lane * 4 * 64, &maps.rope_row, rcol0, r[0], r[1], r[2], r[3], fb);
           }
           __syncwarp();
         }
@@ -436,26 +471,36 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       constexpr uint32_t idS = idesc_bf16_f32(128, 64, 0, 0);
       constexpr uint32_t idO = idesc_bf16_f32(128, 256, 0, 1);
-      // S for tile kk into the (single) S buffer.
+      // S for tile kk into S buffer kk % 2: K-step ks < 16 contracts columns
+      // [16 ks, 16 ks + 16) of the four output-column boxes (A = Q in TMEM),
+      // ks = 16, 17 the two halves of the rope box (A = Q rope in shared
+      // memory). A descriptor plus (byte offset >> 4) describes the same layout
+      // at that offset.
+      const uint64_t dq = smem_desc_noswz(qrope, kQRopeLbo, kQRopeSbo);
       auto issue_s = [&](int kk) {
         const uint32_t sb = stage_base + (kk % kStages) * kStageBytes;
+        const uint32_t sd = tmem + kTmemS + 64u * (uint32_t)(kk & 1);
+        const uint64_t d0 = smem_desc_sw128(sb, 16, 1024);
+        const uint64_t dr = smem_desc_sw64(sb + kRopeOff, 512);
 #pragma unroll
-        for (int ks = 0; ks < kSSteps; ++ks) {
-          const int c = (crank ? 32 : 0) + 16 * ks;  // column relative to col0
-          const uint32_t baddr = sb + (c >> 6) * kBoxBytes + (c & 63) * 2;
-          mma_tmem_a(tmem + kTmemS, tmem + kTmemQ + 8 * ks, smem_desc_sw128(baddr, 16, 1024), idS, ks > 0 ? 1u : 0u);
+        for (int ks = 0; ks < 16; ++ks) {
+          const uint32_t off = (uint32_t)((ks >> 2) * kBoxBytes + (ks & 3) * 32);
+          mma_tmem_a(sd, tmem + kTmemQ + 8 * ks, d0 + (off >> 4), idS, ks > 0 ? 1u : 0u);
         }
-        mma_commit(smem_addr(&misc->s_full));
+        mma_ss(sd, dq, dr, idS, 1u);
+        mma_ss(sd, dq + ((2 * kQRopeLbo) >> 4), dr + (32 >> 4), idS, 1u);
+        mma_commit(smem_addr(&misc->s_full[kk & 1]));
       };
       // O (+)= P V for tile kk; releases the P buffer (in both CTAs) and the stage.
       auto issue_pv = [&](int kk, bool first) {
         const int s = kk % kStages;
-        const uint32_t vb = stage_base + s * kStageBytes;
-        const uint32_t pb = pbuf + (kk & 1) * kPSlotBytes;
-#pragma unroll
-        for (int u = 0; u < 4; ++u)
-          mma_ss(tmem + kTmemO, smem_desc_sw128(pb + 32 * u, 16, 1024), smem_desc_sw128(vb + u * 2048, kBoxBytes, 1024),
-                 idO, (first && u == 0) ? 0u : 1u);
+        const uint64_t dv = smem_desc_sw128(stage_base + s * kStageBytes, kBoxBytes, 1024);
+        const uint64_t dp = smem_desc_sw128(pbuf + (kk & 1) * kPSlotBytes, 16, 1024);
+        // K-step u: P advances 32 B along its swizzled rows, V 16 rows (2048 B)
+        mma_ss(tmem + kTmemO, dp, dv, idO, first ? 0u : 1u);
+        mma_ss(tmem + kTmemO, dp + (32 >> 4), dv + (2048 >> 4), idO, 1u);
+        mma_ss(tmem + kTmemO, dp + (64 >> 4), dv + (4096 >> 4), idO, 1u);
+        mma_ss(tmem + kTmemO, dp + (96 >> 4), dv + (6144 >> 4), idO, 1u);
         mma_commit_cluster(smem_addr(&misc->p_free[kk & 1]), (uint16_t)0x3);
         mma_commit(smem_addr(&misc->empty[s]));
       };
@@ -468,19 +513,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         // PV(kk) needs both CTAs' P of tile kk (and, for the first tile of a
         // task, the previous task's epilogue done with O).
         int ns = 0, np = 0;
-        uint64_t t0 = global_timer_ns();
+        uint64_t t0 = 0;  // start of the current stretch without progress (0: none)
         while (np < n) {
           bool progress = false;
-          if (ns < n) {
-            const int kk = k + ns;
-            if (mbar_test_wait(smem_addr(&misc->full[kk % kStages]), (kk / kStages) & 1) &&
-                (kk == 0 || mbar_test_wait(smem_addr(&misc->s_free), (kk - 1) & 1))) {
-              tc_fence_after();
-              issue_s(kk);
-              ++ns;
-              progress = true;
-            }
-          }
+          // PV first: an S issued ahead of a ready PV delays it by a whole S
           if (np < ns) {
             const int kk = k + np;
             if (mbar_test_wait(smem_addr(&misc->p_full[kk & 1]), (kk >> 1) & 1) &&
@@ -491,15 +527,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
               progress = true;
             }
           }
+          if (ns < n) {
+            const int kk = k + ns;
+            if (mbar_test_wait(smem_addr(&misc->full[kk % kStages]), (kk / kStages) & 1) &&
+                (kk < 2 || mbar_test_wait(smem_addr(&misc->s_free[kk & 1]), ((kk >> 1) & 1) ^ 1))) {
+              tc_fence_after();
+              // all 18 MMAs back to back: the tensor pipe overlaps dependent MMAs
+              // only while they are queued together
+              issue_s(kk);
+              ++ns;
+              progress = true;
+            }
+          }
+          // the clock is read only while nothing is ready (reading it is slow)
           if (progress) {
-            t0 = global_timer_ns();
+            t0 = 0;
           } else if (W.aborted()) {
             ok = false;
             break;
-          } else if (global_timer_ns() - t0 > kTimeoutNs) {
-            W.fail();
-            ok = false;
-            break;
+          } else {
+            const uint64_t now = global_timer_ns();
+            if (t0 == 0) {
+              t0 = now;
+            } else if (now - t0 > kTimeoutNs) {
+              W.fail();
+              ok = false;
+              break;
+            }
           }
         }
         if (!ok) break;
@@ -528,7 +582,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const uint32_t stat_peer =
         map_to_rank(statbuf, peer) + (uint32_t)(quad * kStatQuadBytes) + (uint32_t)rl * 16u;
     const uint32_t xoff = (uint32_t)(quad * kXQuadBytes) + (uint32_t)lane * 16u;
-    const uint32_t xbytes = n_active * (uint32_t)kXQuadBytes;
+    const uint32_t xbytes = n_active * (uint32_t)(kXQuadBytes + kXExpBytes);
+    const uint32_t xexp = xbuf + kXExpOff + (uint32_t)(quad * kXExpBytes) + (uint32_t)rl * 4u;
     int k = 0, j = 0;
 
     while (cur.next(task, pg0, pg1, split)) {
@@ -540,37 +595,37 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const int xs = k & 1;
         // own partial scores of this tile (this thread: its row, tokens 32*th..+31)
         uint32_t own[32];
-        if (!W.wait_warp(&misc->s_full, k & 1)) goto softmax_done;
+        if (!W.wait_warp(&misc->s_full[k & 1], (k >> 1) & 1)) goto softmax_done;
         tc_fence_after();
-        tmem_ld_16x32bx2_32<32>(own_lanes + kTmemS, own);
+        tmem_ld_16x32bx2_32<32>(own_lanes + kTmemS + 64u * (uint32_t)(k & 1), own);
         tmem_wait_ld();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(smem_addr(&misc->s_free));
+        if (lane == 0) mbar_arrive(smem_addr(&misc->s_free[k & 1]));
         // the peer's partial scores of these rows
-        if (expect_thread) mbar_arrive_expect_tx(smem_addr(&misc->x_full[xs]), xbytes);
-        if (!W.wait_warp(&misc->x_full[xs], (k >> 1) & 1)) goto softmax_done;
+        if (expect_thread) mbar_arrive_expect_tx(smem_addr(&misc->x_full), xbytes);
+        if (!W.wait_warp(&misc->x_full, k & 1)) goto softmax_done;
         float sc[32];
         {
-          uint32_t w[24];
+          uint32_t w[16];
 #pragma unroll
-          for (int c = 0; c < 6; ++c) {
-            const uint4 v = ld_shared_v4(xbuf + xs * kXBytes + xoff + c * 512);
+          for (int c = 0; c < 4; ++c) {
+            const uint4 v = ld_shared_v4(xbuf + xoff + c * 512);
             w[4 * c + 0] = v.x;
             w[4 * c + 1] = v.y;
             w[4 * c + 2] = v.z;
             w[4 * c + 3] = v.w;
           }
+          const float inv = fx16_inv(ld_shared_u32(xexp));
+          const float bias = fx16_bias(inv);
 #pragma unroll
-          for (int g = 0; g < 8; ++g) {
-            float f[4];
-            unpack24x4(w[3 * g], w[3 * g + 1], w[3 * g + 2], f);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) sc[4 * g + e] = __uint_as_float(own[4 * g + e]) + f[e];
+          for (int c = 0; c < 16; ++c) {
+            sc[2 * c] = __uint_as_float(own[2 * c]) + fx16_lo(w[c], inv, bias);
+            sc[2 * c + 1] = __uint_as_float(own[2 * c + 1]) + fx16_hi(w[c], inv, bias);
           }
         }
         __syncwarp();
-        if (lane == 0) mbar_arrive(smem_addr(&misc->x_read[xs]));
+        if (lane == 0) mbar_arrive(smem_addr(&misc->x_read));
 
         // mask (written by the producer before the stage's full barrier)
         if (!W.wait_warp(&misc->full[s], (k / kStages) & 1)) goto softmax_done;
@@ -674,50 +729,84 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     if (!W.aborted())
       for (int kk = max(0, k - 2); kk < k; ++kk) W.wait_cluster(&misc->p_free[kk & 1], (kk >> 1) & 1);
     __syncwarp();
-  } else if (warp >= 6) {
-    // ------------------------------------------------------------ helper (rows the peer owns)
+  } else if (warp >= 6 && warp <= 9) {
+    // ------------------------------------------------------------ sender (rows the peer owns)
     const bool lead = (quad == 0 && lane == 0);  // warp 8, lane 0: expects and relays
-    const uint32_t xfull_peer = map_to_rank(smem_addr(&misc->x_full[0]), peer);
-    const uint32_t xempty_peer = map_to_rank(smem_addr(&misc->x_empty[0]), peer);
+    const uint32_t xfull_peer = map_to_rank(smem_addr(&misc->x_full), peer);
+    const uint32_t xempty_peer = map_to_rank(smem_addr(&misc->x_empty), peer);
     const uint32_t xbuf_peer = map_to_rank(xbuf, peer) + (uint32_t)(quad * kXQuadBytes) + (uint32_t)lane * 16u;
+    const uint32_t xexp_peer = map_to_rank(xbuf, peer) + kXExpOff + (uint32_t)(quad * kXExpBytes) + (uint32_t)rl * 4u;
     const uint32_t xdummy_peer = map_to_rank(smem_addr(&misc->xdummy[quad]), peer);
+    int k = 0;
+    bool ok = true;
+
+    // This CTA's softmax warps have read the score slot for tile kk: tell the
+    // peer (their arrives released the reads; this wait acquires them).
+    auto relay_read = [&](int kk) -> bool {
+      if (quad != 0) return true;
+      if (!W.wait_warp(&misc->x_read, kk & 1)) return false;
+      if (lane == 0) st_async_b32(xdummy_peer, (uint32_t)kk, xempty_peer);
+      return true;
+    };
+    // Partial scores of tile kk for the rows the peer owns -> the peer's slot.
+    // The relay for tile kk - 1 goes out before the wait for the peer's relay
+    // of the same tile: with one slot per CTA, the reverse order deadlocks.
+    auto send_s = [&](int kk) -> bool {
+      if (!W.wait_warp(&misc->s_full[kk & 1], (kk >> 1) & 1)) return false;
+      tc_fence_after();
+      uint32_t sr[32];
+      tmem_ld_16x32bx2_32<32>(peer_lanes + kTmemS + 64u * (uint32_t)(kk & 1), sr);
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_addr(&misc->s_free[kk & 1]));
+      // 16-bit fixed point with the row's exponent; masked tokens (any value,
+      // even NaN) neither set the scale nor matter after the receiver masks them
+      const int s = kk % kStages;
+      if (!W.wait_warp(&misc->full[s], (kk / kStages) & 1)) return false;
+      const uint32_t msk = (uint32_t)(misc->stage_mask[s] >> (32 * th));
+      float amax = 0.f;
+#pragma unroll
+      for (int c = 0; c < 32; ++c)
+        if ((msk >> c) & 1u) amax = fmaxf(amax, fabsf(__uint_as_float(sr[c])));
+      amax = fmaxf(amax, __shfl_xor_sync(~0u, amax, 16));
+      const uint32_t ex = fx16_exponent(amax);
+      const float mult = fx16_mult(ex);
+      uint32_t w[16];
+#pragma unroll
+      for (int c = 0; c < 16; ++c) w[c] = fx16_pack2(__uint_as_float(sr[2 * c]), __uint_as_float(sr[2 * c + 1]), mult);
+      if (kk >= 1 && !relay_read(kk - 1)) return false;
+      // the peer's softmax warps have read its slot for tile kk - 1
+      if (kk >= 1 && lead) mbar_arrive_expect_tx(smem_addr(&misc->x_empty), 4u);
+      if (!W.wait_cluster_warp(&misc->x_empty, (kk & 1) ^ 1)) return false;
+      if (quad_active) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          st_async_v4(xbuf_peer + c * 512, w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3], xfull_peer);
+        if (th == 0) st_async_b32(xexp_peer, ex, xfull_peer);
+      }
+      return true;
+    };
+
+    while (ok && cur.next(task, pg0, pg1, split)) {
+      write_q(1);
+      const int n = pg1 - pg0;
+      for (int i = 0; ok && i < n; ++i) ok = send_s(k + i);
+      if (!ok) break;
+      k += n;
+    }
+    if (ok && k > 0) ok = relay_read(k - 1);
+    // the peer relays "slot read" for every score tile sent; collect the last one before exit
+    if (ok) drain_x_empty(k, lead);
+    __syncwarp();
+  } else if (warp >= 10) {
+    // ------------------------------------------------------------ acceptor (rows the peer owns)
+    const bool lead = (quad == 0 && lane == 0);  // warp 12, lane 0: expects the P messages
     const uint32_t pmbytes = n_active * (uint32_t)(kPQuadBytes + kStatQuadBytes);
     int k = 0, j = 0;
     bool ok = true;
     float pm = -INFINITY, pl = 0.f;  // the owner's running max / sum of this thread's row
 
-    // Partial scores of tile kk for the rows the peer owns -> the peer's slot kk % 2.
-    auto send_s = [&](int kk) -> bool {
-      if (!W.wait_warp(&misc->s_full, kk & 1)) return false;
-      tc_fence_after();
-      uint32_t sr[32];
-      tmem_ld_16x32bx2_32<32>(peer_lanes + kTmemS, sr);
-      tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_addr(&misc->s_free));
-      uint32_t w[24];
-#pragma unroll
-      for (int g = 0; g < 8; ++g) pack24x4(&sr[4 * g], &w[3 * g]);
-      const int xs = kk & 1;
-      if (kk >= 2 && lead) mbar_arrive_expect_tx(smem_addr(&misc->x_empty[xs]), 4u);
-      if (!W.wait_cluster_warp(&misc->x_empty[xs], ((kk >> 1) & 1) ^ 1)) return false;
-      if (quad_active) {
-#pragma unroll
-        for (int c = 0; c < 6; ++c)
-          st_async_v4(xbuf_peer + xs * kXBytes + c * 512, w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3],
-                      xfull_peer + 8u * xs);
-      }
-      return true;
-    };
-    // This CTA's softmax warps have read score slot kk % 2: tell the peer
-    // (their arrives released the reads; this wait acquires them).
-    auto relay_read = [&](int kk) -> bool {
-      if (quad != 0) return true;
-      if (!W.wait_warp(&misc->x_read[kk & 1], (kk >> 1) & 1)) return false;
-      if (lane == 0) st_async_b32(xdummy_peer, (uint32_t)kk, xempty_peer + 8u * (kk & 1));
-      return true;
-    };
     // The peer's P of tile kk landed in P buffer kk % 2: rescale the O rows
     // the peer owns by their factor (rare), then release PV(kk).
     auto accept_p = [&](int kk) -> bool {
@@ -742,14 +831,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     };
 
     while (ok && cur.next(task, pg0, pg1, split)) {
-      write_q(1);
       const int n = pg1 - pg0;
-      ok = send_s(k);
-      for (int i = 0; ok && i < n; ++i) {
-        if (i + 1 < n) ok = send_s(k + i + 1);
-        if (ok) ok = relay_read(k + i);
-        if (ok) ok = accept_p(k + i);
-      }
+      for (int i = 0; ok && i < n; ++i) ok = accept_p(k + i);
       if (!ok) break;
       k += n;
       // ------------------------------------------------------------ epilogue (rows the peer owns)
@@ -766,8 +849,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       if (lane == 0) mbar_arrive(smem_addr(&misc->o_empty));
       ++j;
     }
-    // the peer relays "slot read" for every score tile sent; collect the last ones before exit
-    if (ok) drain_tokens(misc->x_empty, k, 4u, lead);
     __syncwarp();
   }
 
@@ -787,9 +868,9 @@ const void* decode_kernel_ptr() { return reinterpret_cast<const void*>(&dec::mla
 int decode_smem_bytes() { return dec::kSmemBytes; }
 int decode_threads() { return dec::kThreads; }
 
-cudaError_t launch_decode(const CUtensorMap& tm_tile, const CUtensorMap& tm_row, const DecodeArgs& args, int workers,
+cudaError_t launch_decode(const CacheMaps& maps, const DecodeArgs& args, int workers,
                           cudaStream_t stream) {
-  dec::mla_decode_kernel<<<2 * workers, dec::kThreads, dec::kSmemBytes, stream>>>(tm_tile, tm_row, args);
+  dec::mla_decode_kernel<<<2 * workers, dec::kThreads, dec::kSmemBytes, stream>>>(maps, args);
   return cudaGetLastError();
 }
 

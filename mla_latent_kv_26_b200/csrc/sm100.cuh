@@ -163,6 +163,11 @@ MLA_DEV void bulk_copy_to_cta(uint32_t dst_cluster, uint32_t src_cta, uint32_t b
                : "memory");
 }
 
+MLA_DEV uint32_t ld_shared_u32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
+}
 MLA_DEV uint4 ld_shared_v4(uint32_t addr) {
   uint4 v;
   asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
@@ -194,6 +199,21 @@ MLA_DEV void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;"
 MLA_DEV uint64_t smem_desc_sw128(uint32_t addr, uint32_t lbo, uint32_t sbo) {
   return (uint64_t)((addr & 0x3FFFFu) >> 4) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
          ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
+}
+
+// Shared-memory matrix descriptor, 64-byte swizzle, K-major: rows of 64 B,
+// `sbo` = stride between 8-row groups.
+MLA_DEV uint64_t smem_desc_sw64(uint32_t addr, uint32_t sbo) {
+  return (uint64_t)((addr & 0x3FFFFu) >> 4) | (1ull << 16) | ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) |
+         (4ull << 61);
+}
+
+// Shared-memory matrix descriptor, no swizzle, K-major: 8x16-byte core
+// matrices; `lbo` = bytes between core matrices adjacent in K, `sbo` = bytes
+// between 8-row groups.
+MLA_DEV uint64_t smem_desc_noswz(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+  return (uint64_t)((addr & 0x3FFFFu) >> 4) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+         ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46);
 }
 
 // Instruction descriptor, kind::f16: bf16 A and B, fp32 accumulator.
@@ -327,6 +347,31 @@ MLA_DEV float ex2(float x) {
 // 24-bit floats: an fp32 bit pattern rounded (half up in magnitude) to its
 // top three bytes (sign, exponent, 15 mantissa bits; relative error <= 2^-16).
 // Four of them pack into three words, byte-wise little endian.
+// 16-bit block fixed point (one power-of-two scale per row of 64 values):
+// with E the biased exponent of the row's largest magnitude (at least 15),
+// q = round(x * 2^(141 - E)) lies in [-32767, 32767] and x = q * 2^(E - 141),
+// so the absolute error is at most 2^(E - 142) <= max|x| * 2^-15.
+MLA_DEV uint32_t fx16_exponent(float amax) { return max((__float_as_uint(amax) >> 23) & 0xFFu, 15u); }
+MLA_DEV float fx16_mult(uint32_t e) { return __uint_as_float((268u - e) << 23); }  // 2^(141 - e)
+MLA_DEV float fx16_inv(uint32_t e) { return __uint_as_float((e - 14u) << 23); }    // 2^(e - 141)
+// Two values -> q + 32768 in the low and high halves: the sum with
+// 1.5 * 2^23 + 2^15 has unit spacing, so its low 16 bits are round(x m) + 2^15.
+MLA_DEV uint32_t fx16_pack2(float a, float b, float mult) {
+  constexpr float kMagic = 12615680.0f, kLo = kMagic - 32767.0f, kHi = kMagic + 32767.0f;
+  const float x = fminf(fmaxf(fmaf(a, mult, kMagic), kLo), kHi);
+  const float y = fminf(fmaxf(fmaf(b, mult, kMagic), kLo), kHi);
+  return __byte_perm(__float_as_uint(x), __float_as_uint(y), 0x5410);
+}
+// q * inv from the low / high half: 2^23 + (q + 2^15) is built by a byte
+// permute, and (2^23 + u) * inv - (2^23 + 2^15) * inv is exact in one FMA.
+MLA_DEV float fx16_bias(float inv) { return -8421376.0f * inv; }
+MLA_DEV float fx16_lo(uint32_t w, float inv, float bias) {
+  return fmaf(__uint_as_float(__byte_perm(w, 0x4B000000u, 0x7410)), inv, bias);
+}
+MLA_DEV float fx16_hi(uint32_t w, float inv, float bias) {
+  return fmaf(__uint_as_float(__byte_perm(w, 0x4B000000u, 0x7432)), inv, bias);
+}
+
 MLA_DEV void pack24x4(const uint32_t* f, uint32_t* w) {
   const uint32_t r0 = f[0] + 0x80u, r1 = f[1] + 0x80u, r2 = f[2] + 0x80u, r3 = f[3] + 0x80u;
   w[0] = __byte_perm(r0, r1, 0x5321);  // r0.b1 r0.b2 r0.b3 r1.b1
