@@ -749,9 +749,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       return true;
     };
     // Partial scores of tile kk for the rows the peer owns -> the peer's slot.
-    // The relay for tile kk - 1 goes out before the wait for the peer's relay
-    // of the same tile: with one slot per CTA, the reverse order deadlocks.
+    // The relay for tile kk - 1 goes out first: it must precede the wait for
+    // the peer's relay of the same tile (with one slot per CTA, the reverse
+    // order deadlocks), and sending it before the S wait keeps the peer's
+    // score send from waiting on this CTA's S.
     auto send_s = [&](int kk) -> bool {
+      if (kk >= 1 && !relay_read(kk - 1)) return false;
       if (!W.wait_warp(&misc->s_full[kk & 1], (kk >> 1) & 1)) return false;
       tc_fence_after();
       uint32_t sr[32];
@@ -775,7 +778,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       uint32_t w[16];
 #pragma unroll
       for (int c = 0; c < 16; ++c) w[c] = fx16_pack2(__uint_as_float(sr[2 * c]), __uint_as_float(sr[2 * c + 1]), mult);
-      if (kk >= 1 && !relay_read(kk - 1)) return false;
       // the peer's softmax warps have read its slot for tile kk - 1
       if (kk >= 1 && lead) mbar_arrive_expect_tx(smem_addr(&misc->x_empty), 4u);
       if (!W.wait_cluster_warp(&misc->x_empty, (kk & 1) ^ 1)) return false;
