@@ -272,14 +272,26 @@ def main():
     dec = decoder_for(inp, num_sms=args.num_sms, device=dev)
     stream = torch.cuda.current_stream(dev)
 
-    def step(ev=None):
-        dec.plan_step(g["seq_lens"], stream)
+    # ev: events recorded before plan, before decode, after decode, after combine
+    def step(ev=None, st=None):
+        st = stream if st is None else st
         if ev is not None:
-            ev[0].record(stream)
-        dec.decode_step(g["q"], g["cache"], g["block_table"], g["seq_lens"], g["indices"], stream)
+            ev[0].record(st)
+        dec.plan_step(g["seq_lens"], st)
         if ev is not None:
-            ev[1].record(stream)
-        dec.combine_step(stream)
+            ev[1].record(st)
+        dec.decode_step(g["q"], g["cache"], g["block_table"], g["seq_lens"], g["indices"], st)
+        if ev is not None:
+            ev[2].record(st)
+        dec.combine_step(st)
+        if ev is not None:
+            ev[3].record(st)
+
+    # Inputs within twice the L2 size are flushed from L2 before every timed
+    # step (a write of a buffer twice the L2 size, outside the step's events).
+    l2_bytes = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush_l2 = acc["bytes"] < 2 * l2_bytes
+    flush_buf = torch.empty(2 * l2_bytes, dtype=torch.uint8, device=dev) if flush_l2 else None
 
     def barrier():
         if world > 1:
@@ -293,7 +305,7 @@ def main():
         raise RuntimeError(f"device error after warm-up: status {st} bits {bits:#x}")
 
     K = args.steps
-    kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    kev = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(4)) for _ in range(K)]
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     sampler = ClockSampler(local) if not args.profile else None
     barrier()
@@ -302,18 +314,23 @@ def main():
         sampler.__enter__()
     t_start.record(stream)
     for i in range(K):
+        if flush_l2:
+            flush_buf.fill_(i & 0xFF)
         step(kev[i])
     t_end.record(stream)
     torch.cuda.synchronize(dev)
     if sampler:
         sampler.__exit__(None, None, None)
     barrier()
-    elapsed_ms = t_start.elapsed_time(t_end)
-    decode_ms = sum(a.elapsed_time(b) for a, b in kev) / K
-    tmax = torch.tensor([elapsed_ms, decode_ms], dtype=torch.float64, device=dev)
+    # with the L2 flush, the timed work is the sum of the steps' own intervals
+    elapsed_ms = sum(e[0].elapsed_time(e[3]) for e in kev) if flush_l2 else t_start.elapsed_time(t_end)
+    plan_ms = sum(e[0].elapsed_time(e[1]) for e in kev) / K
+    decode_ms = sum(e[1].elapsed_time(e[2]) for e in kev) / K
+    combine_ms = sum(e[2].elapsed_time(e[3]) for e in kev) / K
+    tmax = torch.tensor([elapsed_ms, decode_ms, plan_ms, combine_ms], dtype=torch.float64, device=dev)
     if world > 1:
         dist.all_reduce(tmax, op=dist.ReduceOp.MAX)
-    elapsed_ms, decode_ms = float(tmax[0]), float(tmax[1])
+    elapsed_ms, decode_ms, plan_ms, combine_ms = (float(x) for x in tmax)
     ms_per_step = elapsed_ms / K
 
     if args.profile:
@@ -362,6 +379,33 @@ def main():
     if st != 0:
         raise RuntimeError(f"device error in timed region: status {st} bits {bits:#x}")
 
+    # small inputs: the same step captured in a CUDA graph (launch overhead removed), L2 flushed before each replay
+    graph_ms = None
+    if flush_l2:
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(stream)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(side):
+            step(st=side)  # warm the capture stream
+            with torch.cuda.graph(graph, stream=side):
+                step(st=side)
+        stream.wait_stream(side)
+        gev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+        barrier()
+        torch.cuda.synchronize(dev)
+        for i in range(K):
+            flush_buf.fill_(i & 0xFF)
+            gev[i][0].record(stream)
+            graph.replay()
+            gev[i][1].record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+        gms = torch.tensor([sum(a.elapsed_time(b) for a, b in gev) / K], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(gms, op=dist.ReduceOp.MAX)
+        graph_ms = float(gms)
+        del graph
+
     peaks, peak_src = load_peaks()
     t_hbm = acc["bytes"] / (peaks["hbm_gbs"] * 1e9)
     t_tc = acc["flops"] / (peaks["bf16_tflops"] * 1e12)
@@ -396,14 +440,17 @@ def main():
                    "kv_len": f"{w.len_lo}..{w.len_hi}" + (f" top{w.topk}" if w.topk else ""),
                    "kv_tokens_per_step": acc["kv_tokens"], "bytes_per_step": acc["bytes"],
                    "flops_per_step": acc["flops"], "seed": w.seed, "workers": dec.num_workers,
-                   "l2": f"inputs larger than L2 ({acc['bytes'] / 1e6:.0f} MB read per step), no flush"
-                   if acc["bytes"] > 256e6 else "inputs smaller than L2: not flushed",
+                   "l2": (f"{acc['bytes'] / 1e6:.0f} MB read per step, within 2x L2 ({l2_bytes / 1e6:.0f} MB): "
+                          f"L2 flushed by a {2 * l2_bytes / 1e6:.0f} MB write before every timed step")
+                   if flush_l2 else f"inputs larger than 2x L2 ({acc['bytes'] / 1e6:.0f} MB read per step), no flush",
                    "parallelism": f"replicas x{world}"},
         "roofline": roof,
         "e2e": {"value": world * acc["kv_tokens"] / (e2e_ms / 1e3), "unit": UNIT,
                 "h2d_bytes_per_step": acc["h2d_bytes"], "d2h_bytes_per_step": acc["d2h_bytes"],
                 "ms_per_step": e2e_ms},
         "gpu_launches": 3 * K,
+        "kernels_us": {"plan": plan_ms * 1e3, "decode": decode_ms * 1e3, "combine": combine_ms * 1e3},
+        "graph_ms_per_step": graph_ms,
         "clocks": sampler.summary() if sampler else None,
     }
     if rank == 0 and world == 1:
