@@ -228,6 +228,26 @@ def run_reference(args, inp, rank):
     print(json.dumps(line), flush=True)
 
 
+# ---------------------------------------------------------------- ranks
+
+
+def max_over_ranks(values, world: int, device) -> list:
+    """Element-wise maximum of per-rank timings over all ranks (the job is as
+    slow as its slowest rank); identity for a single process."""
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t]
+
+
+def job_value(world: int, kv_tokens: int, ms_per_step: float) -> float:
+    """Whole-job KV tokens per second: every rank decodes its own replica of
+    the step's batch, timed by the slowest rank."""
+    return world * kv_tokens / (ms_per_step / 1e3)
+
+
 # ---------------------------------------------------------------- GPU arm
 
 
@@ -327,10 +347,7 @@ def main():
     plan_ms = sum(e[0].elapsed_time(e[1]) for e in kev) / K
     decode_ms = sum(e[1].elapsed_time(e[2]) for e in kev) / K
     combine_ms = sum(e[2].elapsed_time(e[3]) for e in kev) / K
-    tmax = torch.tensor([elapsed_ms, decode_ms, plan_ms, combine_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(tmax, op=dist.ReduceOp.MAX)
-    elapsed_ms, decode_ms, plan_ms, combine_ms = (float(x) for x in tmax)
+    elapsed_ms, decode_ms, plan_ms, combine_ms = max_over_ranks([elapsed_ms, decode_ms, plan_ms, combine_ms], world, dev)
     ms_per_step = elapsed_ms / K
 
     if args.profile:
@@ -370,10 +387,7 @@ def main():
     e1.record(stream)
     torch.cuda.synchronize(dev)
     barrier()
-    e2e_ms = torch.tensor([e0.elapsed_time(e1) / K2], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
-    e2e_ms = float(e2e_ms)
+    (e2e_ms,) = max_over_ranks([e0.elapsed_time(e1) / K2], world, dev)
 
     st, bits = dec.error(stream)
     if st != 0:
@@ -400,10 +414,7 @@ def main():
             gev[i][1].record(stream)
         torch.cuda.synchronize(dev)
         barrier()
-        gms = torch.tensor([sum(a.elapsed_time(b) for a, b in gev) / K], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(gms, op=dist.ReduceOp.MAX)
-        graph_ms = float(gms)
+        (graph_ms,) = max_over_ranks([sum(a.elapsed_time(b) for a, b in gev) / K], world, dev)
         del graph
 
     peaks, peak_src = load_peaks()
@@ -430,7 +441,7 @@ def main():
     roof["tflop_per_s"] = achieved_tf
     roof["tensor_frac"] = achieved_tf / peaks["bf16_tflops"]
 
-    value = world * acc["kv_tokens"] / (ms_per_step / 1e3)
+    value = job_value(world, acc["kv_tokens"], ms_per_step)
     w = inp["workload"]
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
@@ -445,7 +456,7 @@ def main():
                    if flush_l2 else f"inputs larger than 2x L2 ({acc['bytes'] / 1e6:.0f} MB read per step), no flush",
                    "parallelism": f"replicas x{world}"},
         "roofline": roof,
-        "e2e": {"value": world * acc["kv_tokens"] / (e2e_ms / 1e3), "unit": UNIT,
+        "e2e": {"value": job_value(world, acc["kv_tokens"], e2e_ms), "unit": UNIT,
                 "h2d_bytes_per_step": acc["h2d_bytes"], "d2h_bytes_per_step": acc["d2h_bytes"],
                 "ms_per_step": e2e_ms},
         "gpu_launches": 3 * K,
