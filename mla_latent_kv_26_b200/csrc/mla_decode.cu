@@ -590,14 +590,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       write_q(0);
       float m_run = -INFINITY, l_run = 0.f;
       const int ntiles = pg1 - pg0;
+      // own partial scores of the current tile (this thread: its row, tokens
+      // 32*th..+31); the next tile's are loaded at the end of this one when
+      // they are already complete, so the TMEM read overlaps the tile's tail
+      uint32_t own[32];
+      bool own_loading = false;
       for (int i = 0; i < ntiles; ++i, ++k) {
         const int s = k % kStages;
         const int xs = k & 1;
-        // own partial scores of this tile (this thread: its row, tokens 32*th..+31)
-        uint32_t own[32];
-        if (!W.wait_warp(&misc->s_full[k & 1], (k >> 1) & 1)) goto softmax_done;
-        tc_fence_after();
-        tmem_ld_16x32bx2_32<32>(own_lanes + kTmemS + 64u * (uint32_t)(k & 1), own);
+        if (!own_loading) {
+          if (!W.wait_warp(&misc->s_full[k & 1], (k >> 1) & 1)) goto softmax_done;
+          tc_fence_after();
+          tmem_ld_16x32bx2_32<32>(own_lanes + kTmemS + 64u * (uint32_t)(k & 1), own);
+        }
+        own_loading = false;
         tmem_wait_ld();
         tc_fence_before();
         __syncwarp();
@@ -708,6 +714,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_addr(&misc->p_full[xs]));
+        if (i + 1 < ntiles &&
+            __all_sync(~0u, mbar_test_wait(smem_addr(&misc->s_full[(k + 1) & 1]), ((k + 1) >> 1) & 1))) {
+          tc_fence_after();
+          tmem_ld_16x32bx2_32<32>(own_lanes + kTmemS + 64u * (uint32_t)((k + 1) & 1), own);
+          own_loading = true;
+        }
       }
 
       // ------------------------------------------------------------ epilogue (owned rows)
