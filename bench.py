@@ -325,9 +325,12 @@ def main():
         raise RuntimeError(f"device error after warm-up: status {st} bits {bits:#x}")
 
     K = args.steps
-    kev = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(4)) for _ in range(K)]
-    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     sampler = ClockSampler(local) if not args.profile else None
+
+    # Loop A (the headline): K steps with events only at step boundaries, so
+    # the plan, decode and combine launches overlap as they do for a caller.
+    sev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize(dev)
     if sampler:
@@ -336,14 +339,29 @@ def main():
     for i in range(K):
         if flush_l2:
             flush_buf.fill_(i & 0xFF)
-        step(kev[i])
+            sev[i][0].record(stream)
+        step()
+        if flush_l2:
+            sev[i][1].record(stream)
     t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    # with the L2 flush, the timed work is the sum of the steps' own intervals
+    elapsed_ms = sum(a.elapsed_time(b) for a, b in sev) if flush_l2 else t_start.elapsed_time(t_end)
+
+    # Loop B: K more steps with an event between every two kernels, for each
+    # kernel's own time (the decode kernel's is the roofline's denominator).
+    kev = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(4)) for _ in range(K)]
+    barrier()
+    torch.cuda.synchronize(dev)
+    for i in range(K):
+        if flush_l2:
+            flush_buf.fill_(i & 0xFF)
+        step(kev[i])
     torch.cuda.synchronize(dev)
     if sampler:
         sampler.__exit__(None, None, None)
     barrier()
-    # with the L2 flush, the timed work is the sum of the steps' own intervals
-    elapsed_ms = sum(e[0].elapsed_time(e[3]) for e in kev) if flush_l2 else t_start.elapsed_time(t_end)
     plan_ms = sum(e[0].elapsed_time(e[1]) for e in kev) / K
     decode_ms = sum(e[1].elapsed_time(e[2]) for e in kev) / K
     combine_ms = sum(e[2].elapsed_time(e[3]) for e in kev) / K
@@ -357,41 +375,67 @@ def main():
             dist.destroy_process_group()
         return
 
-    # ---- end to end through the public API with pinned host buffers
+    # ---- end to end through the public API with pinned host buffers: every
+    # step copies its inputs in and its output and LSE back. Consecutive steps
+    # alternate between two decoders on two streams, so one step's copies
+    # overlap the neighbouring steps' kernels (as a caller decoding step after
+    # step would run it); each stream keeps its own device buffers.
     host_in = {k: inp[k].pin_memory() for k in ("q", "block_table", "seq_lens")}
     if inp["indices"] is not None:
         host_in["indices"] = inp["indices"].pin_memory()
-    host_out = torch.empty(dec.out.shape, dtype=dec.out.dtype).pin_memory()
-    host_lse = torch.empty(dec.lse.shape, dtype=dec.lse.dtype).pin_memory()
-    dev_in = {k: torch.empty_like(v, device=dev) for k, v in host_in.items()}
+    lanes = []
+    for li in range(2):
+        dl = dec if li == 0 else decoder_for(inp, num_sms=args.num_sms, device=dev)
+        lanes.append({
+            "dec": dl,
+            "stream": torch.cuda.Stream(dev),
+            "dev_in": {k: torch.empty_like(v, device=dev) for k, v in host_in.items()},
+            "host_out": torch.empty(dl.out.shape, dtype=dl.out.dtype).pin_memory(),
+            "host_lse": torch.empty(dl.lse.shape, dtype=dl.lse.dtype).pin_memory(),
+        })
 
-    def e2e_step():
-        for k, v in host_in.items():
-            dev_in[k].copy_(v, non_blocking=True)
-        dec.plan_step(dev_in["seq_lens"], stream)
-        dec.decode_step(dev_in["q"], g["cache"], dev_in["block_table"], dev_in["seq_lens"], dev_in.get("indices"),
-                        stream)
-        dec.combine_step(stream)
-        host_out.copy_(dec.out, non_blocking=True)
-        host_lse.copy_(dec.lse, non_blocking=True)
+    def e2e_step(i):
+        ln = lanes[i % len(lanes)]
+        st, dl, din = ln["stream"], ln["dec"], ln["dev_in"]
+        with torch.cuda.stream(st):
+            for k, v in host_in.items():
+                din[k].copy_(v, non_blocking=True)
+            dl.plan_step(din["seq_lens"], st)
+            dl.decode_step(din["q"], g["cache"], din["block_table"], din["seq_lens"], din.get("indices"), st)
+            dl.combine_step(st)
+            ln["host_out"].copy_(dl.out, non_blocking=True)
+            ln["host_lse"].copy_(dl.lse, non_blocking=True)
 
-    for _ in range(args.warmup):
-        e2e_step()
+    def lanes_wait(ev):
+        for ln in lanes:
+            ln["stream"].wait_event(ev)
+
+    def join_lanes():
+        for ln in lanes:
+            stream.wait_stream(ln["stream"])
+
+    torch.cuda.synchronize(dev)
+    for i in range(args.warmup):
+        e2e_step(i)
+    torch.cuda.synchronize(dev)
     K2 = max(3, min(K, 50))
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize(dev)
     e0.record(stream)
-    for _ in range(K2):
-        e2e_step()
+    lanes_wait(e0)
+    for i in range(K2):
+        e2e_step(i)
+    join_lanes()
     e1.record(stream)
     torch.cuda.synchronize(dev)
     barrier()
     (e2e_ms,) = max_over_ranks([e0.elapsed_time(e1) / K2], world, dev)
 
-    st, bits = dec.error(stream)
-    if st != 0:
-        raise RuntimeError(f"device error in timed region: status {st} bits {bits:#x}")
+    for ln in lanes:
+        st, bits = ln["dec"].error(stream)
+        if st != 0:
+            raise RuntimeError(f"device error in timed region: status {st} bits {bits:#x}")
 
     # small inputs: the same step captured in a CUDA graph (launch overhead removed), L2 flushed before each replay
     graph_ms = None
@@ -458,7 +502,9 @@ def main():
         "roofline": roof,
         "e2e": {"value": job_value(world, acc["kv_tokens"], e2e_ms), "unit": UNIT,
                 "h2d_bytes_per_step": acc["h2d_bytes"], "d2h_bytes_per_step": acc["d2h_bytes"],
-                "ms_per_step": e2e_ms},
+                "ms_per_step": e2e_ms, "streams": len(lanes),
+                "note": "plan + decode + combine through the C ABI, inputs from pinned host memory and out/lse "
+                        "back every step; consecutive steps alternate between two decoders on two streams"},
         "gpu_launches": 3 * K,
         "kernels_us": {"plan": plan_ms * 1e3, "decode": decode_ms * 1e3, "combine": combine_ms * 1e3},
         "graph_ms_per_step": graph_ms,
