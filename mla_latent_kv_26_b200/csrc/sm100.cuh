@@ -1,7 +1,8 @@
 // Thin inline-PTX wrappers for the sm_100a features the decode kernel uses:
-// mbarriers (with bounded waits), TMA tile and gather4 loads, cluster/DSMEM
-// access, asynchronous remote stores, and tcgen05 (TMEM allocation, MMA,
-// commit, loads/stores, fences). Written from the public PTX ISA.
+// mbarriers, TMA tile and gather4 loads, cluster/DSMEM access (asynchronous
+// remote stores, bulk copies), tcgen05 (TMEM allocation, MMA, commit,
+// loads/stores, fences), and the 16-bit block fixed-point packing of the
+// score exchange. Written from the public PTX ISA.
 #pragma once
 
 #include <cuda.h>
@@ -43,9 +44,6 @@ MLA_DEV void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
-MLA_DEV void named_barrier(uint32_t id, uint32_t nthreads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
 
 // ---------------------------------------------------------------- mbarrier
 
@@ -59,10 +57,6 @@ MLA_DEV void mbar_arrive(uint32_t bar) {
 }
 MLA_DEV void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
-}
-// Arrive on a barrier in another CTA of the cluster (address from map_to_rank).
-MLA_DEV void mbar_arrive_remote(uint32_t cluster_bar) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar) : "memory");
 }
 
 MLA_DEV bool mbar_try_wait(uint32_t bar, uint32_t parity) {
@@ -258,24 +252,6 @@ MLA_DEV void mma_commit(uint32_t bar) {
 MLA_DEV void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 MLA_DEV void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
-// 32 lanes x 32 consecutive 32-bit columns (each thread: its lane, 32 columns).
-MLA_DEV void tmem_ld_32(uint32_t taddr, uint32_t (&r)[32]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
-        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]),
-        "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
-        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-      : "r"(taddr));
-}
-MLA_DEV void tmem_ld_16(uint32_t taddr, uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
-        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-      : "r"(taddr));
-}
 MLA_DEV void tmem_st_32(uint32_t taddr, const uint32_t (&r)[32]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
@@ -285,19 +261,6 @@ MLA_DEV void tmem_st_32(uint32_t taddr, const uint32_t (&r)[32]) {
       "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]),
       "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
       : "memory");
-}
-MLA_DEV void tmem_st_16(uint32_t taddr, const uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
-          taddr),
-      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
-      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
-      : "memory");
-}
-MLA_DEV void tmem_st_8(uint32_t taddr, const uint32_t (&r)[8]) {
-  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"(r[0]),
-               "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
-               : "memory");
 }
 
 
@@ -325,15 +288,6 @@ MLA_DEV void tmem_st_16x32bx2_32(uint32_t taddr, const uint32_t (&r)[32]) {
       "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31]), "n"(kSplit)
       : "memory");
 }
-template <int kSplit>
-MLA_DEV void tmem_st_16x32bx2_16(uint32_t taddr, const uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.16x32bx2.x16.b32 [%0], %17, {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
-          taddr),
-      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
-      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "n"(kSplit)
-      : "memory");
-}
 
 // ---------------------------------------------------------------- math
 
@@ -344,9 +298,6 @@ MLA_DEV float ex2(float x) {
   return y;
 }
 
-// 24-bit floats: an fp32 bit pattern rounded (half up in magnitude) to its
-// top three bytes (sign, exponent, 15 mantissa bits; relative error <= 2^-16).
-// Four of them pack into three words, byte-wise little endian.
 // 16-bit block fixed point (one power-of-two scale per row of 64 values):
 // with E the biased exponent of the row's largest magnitude (at least 15),
 // q = round(x * 2^(141 - E)) lies in [-32767, 32767] and x = q * 2^(E - 141),
@@ -372,19 +323,7 @@ MLA_DEV float fx16_hi(uint32_t w, float inv, float bias) {
   return fmaf(__uint_as_float(__byte_perm(w, 0x4B000000u, 0x7432)), inv, bias);
 }
 
-MLA_DEV void pack24x4(const uint32_t* f, uint32_t* w) {
-  const uint32_t r0 = f[0] + 0x80u, r1 = f[1] + 0x80u, r2 = f[2] + 0x80u, r3 = f[3] + 0x80u;
-  w[0] = __byte_perm(r0, r1, 0x5321);  // r0.b1 r0.b2 r0.b3 r1.b1
-  w[1] = __byte_perm(r1, r2, 0x6532);  // r1.b2 r1.b3 r2.b1 r2.b2
-  w[2] = __byte_perm(r2, r3, 0x7653);  // r2.b3 r3.b1 r3.b2 r3.b3
-}
-MLA_DEV void unpack24x4(uint32_t w0, uint32_t w1, uint32_t w2, float* f) {
-  f[0] = __uint_as_float(w0 << 8);
-  f[1] = __uint_as_float(__byte_perm(w0, w1, 0x5430) & 0xFFFFFF00u);
-  f[2] = __uint_as_float(__byte_perm(w1, w2, 0x4320) & 0xFFFFFF00u);
-  f[3] = __uint_as_float(w2 & 0xFFFFFF00u);
-}
-
+// Two floats -> bf16x2 (round to nearest even), `lo` in the low half.
 MLA_DEV uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
