@@ -80,7 +80,7 @@ typedef enum {
 typedef struct {
   int32_t batch;             /* B >= 0 */
   int32_t q_len;             /* Sq >= 1: new query tokens per sequence (2 = MTP pair) */
-  int32_t num_heads;         /* H: multiple of 16, 16..128 */
+  int32_t num_heads;         /* H: 1..128 */
   int32_t d_latent;          /* must be 512 (kv_lora_rank) */
   int32_t d_rope;            /* must be 64 (qk_rope_head_dim) */
   int32_t page_size;         /* must be 64 tokens */

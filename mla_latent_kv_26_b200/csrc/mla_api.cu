@@ -85,7 +85,7 @@ mla_status_t check_desc(const mla_decode_desc_t* d) {
   if (!(d->softmax_scale > 0.f) || !isfinite(d->softmax_scale)) return MLA_ERR_INVALID_ARG;
   if (d->topk > 0 && d->causal) return MLA_ERR_INVALID_ARG;  // a sparse row's tokens are the listed ones
   if (d->d_latent != kDLatent || d->d_rope != kDRope || d->page_size != kPage) return MLA_ERR_UNSUPPORTED;
-  if (d->num_heads % 16 != 0 || d->num_heads > kMaxHeads) return MLA_ERR_UNSUPPORTED;
+  if (d->num_heads > kMaxHeads) return MLA_ERR_UNSUPPORTED;
   const long long tasks = (long long)d->batch * d->q_len;
   const long long rows = (long long)d->num_pages * kPage;
   if (tasks > (1 << 24) || rows > 0x7fffffffLL || (long long)d->max_pages_per_seq * kPage > 0x7fffffffLL)

@@ -48,8 +48,8 @@ def _desc(libmla, **kw):
     (dict(batch=-1), 1), (dict(q_len=0), 1), (dict(num_pages=0), 1), (dict(max_pages_per_seq=0), 1),
     (dict(topk=-3), 1), (dict(causal=True, topk=4), 1), (dict(softmax_scale=0.0), 1),
     (dict(softmax_scale=float("nan")), 1), (dict(softmax_scale=float("inf")), 1),
-    (dict(d_latent=256), 2), (dict(d_rope=32), 2), (dict(page_size=16), 2), (dict(num_heads=24), 2),
-    (dict(num_heads=256), 2), (dict(num_heads=8), 2),
+    (dict(d_latent=256), 2), (dict(d_rope=32), 2), (dict(page_size=16), 2), (dict(num_heads=0), 1),
+    (dict(num_heads=129), 2), (dict(num_heads=256), 2),
 ])
 def test_bad_descriptors_rejected_before_launch(libmla, kw, status):
     d = _desc(libmla, **kw)
