@@ -25,6 +25,9 @@ Modules:
   and the unabsorbed ("naive") path used to pin the absorbed one.
 * :mod:`oracle.plan` — the split schedule (a1) written as a plain sequential
   definition of a balanced contiguous partition.
+* :mod:`oracle.cache_insert` — the step before decode: kv_norm (RMSNorm) of the
+  latent, the rotary embedding of the rope key, and the write into the token's
+  row of the paged cache.
 
 Pins (tests/test_oracle.py): absorption equivalence against the unabsorbed
 path, single-key exactness, probabilities summing to one, brute force with
@@ -52,3 +55,4 @@ from .decode import (  # noqa: F401
     unabsorbed_attention,
 )
 from .plan import split_plan  # noqa: F401
+from .cache_insert import rms_norm, rope_pairs, cache_insert  # noqa: F401,E402
