@@ -248,6 +248,164 @@ def job_value(world: int, kv_tokens: int, ms_per_step: float) -> float:
     return world * kv_tokens / (ms_per_step / 1e3)
 
 
+# ---------------------------------------------------------------- cache insert (--op insert)
+
+INSERT_METRIC = "MLA latent-cache insert tokens/s (kv_norm + RoPE + paged write) and achieved GB/s vs HBM roofline"
+INSERT_UNIT = "tokens/s"
+
+
+def insert_accounting(d: dict) -> dict:
+    """Algorithmic bytes of one insert: per token its input row (1152 B), its
+    cache row (1152 B), sequence id and position (8 B); per distinct position
+    one cos/sin row (256 B); per distinct (sequence, page) one block-table
+    entry; the weight once."""
+    n = int(d["kv"].shape[0])
+    pos = d["positions"].to(torch.int64)
+    pages = torch.unique(d["seq_ids"].to(torch.int64) * (1 << 32) + pos // 64).numel()
+    bytes_ = n * (2 * 576 * 2 + 8) + torch.unique(pos).numel() * 256 + pages * 4 + 1024
+    return {"tokens": n, "bytes": int(bytes_), "h2d_bytes": n * (576 * 2 + 8), "d2h_bytes": 4}
+
+
+def insert_oracle_sample(d: dict, budget_s: float):
+    """The oracle's insert on the tokens of sequence 0 (one page, 64 tokens, per
+    call; wrapping round to its start) until the budget is used; returns
+    (tokens, seconds)."""
+    import oracle
+
+    t0, done = time.perf_counter(), 0
+    n0 = int((d["seq_ids"] == 0).sum())
+    while time.perf_counter() - t0 < budget_s:
+        i = done % n0
+        k = min(64 - i % 64, n0 - i)
+        base = (i // 64) * 64
+        page = int(d["block_table"][0, i // 64])
+        oracle.cache_insert(d["cache"][page:page + 1], torch.zeros(1, 1, dtype=torch.int32),
+                            torch.zeros(k, dtype=torch.int32), d["positions"][i:i + k] - base, d["kv"][i:i + k],
+                            d["weight"], 1e-6, d["cos"][base:], d["sin"][base:])
+        done += k
+    return done, time.perf_counter() - t0
+
+
+def run_insert_bench(args, world, rank, local):
+    from mla_latent_kv_26_b200.workloads import insert_inputs
+
+    B, T = args.insert_batch, args.insert_tokens
+    d = insert_inputs(lens=[T] * B, new_tokens=[T] * B, seed=5)
+    acc = insert_accounting(d)
+    name = f"insert-b{B}-prefill{T}"
+    cfg = {"workload": f"{name}: {B} sequences x {T} new tokens (positions 0..{T - 1}), 576-wide rows",
+           "tokens_per_step": acc["tokens"], "bytes_per_step": acc["bytes"]}
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        torch.set_num_threads(os.cpu_count() or 1)
+        secs, toks = 0.0, 0
+        for s in range(args.warmup + args.steps):
+            n, dt = insert_oracle_sample(d, 0.5)
+            if s >= args.warmup:
+                toks, secs = toks + n, secs + dt
+        v = toks / secs
+        print(json.dumps({
+            "impl": "reference", "metric": INSERT_METRIC, "value": v, "unit": INSERT_UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": cfg,
+            "cpu_baseline": {"value": v, "unit": INSERT_UNIT, "cores": torch.get_num_threads(), "kind": "oracle",
+                             "sample": "float64 oracle insert, about 0.5 s of tokens of sequence 0 per step"},
+            "e2e": {"value": v, "unit": INSERT_UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}), flush=True)
+        return
+
+    import torch.distributed as dist
+
+    from mla_latent_kv_26_b200.decoder import cache_insert
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+    g = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in d.items()}
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(kv, seq, pos, st):
+        cache_insert(kv, g["weight"], g["cos"], g["sin"], seq, pos, g["block_table"], g["cache"], error_word=err,
+                     stream=st)
+
+    # Steady state, no L2 flush: a step reads and writes more than the L2
+    # holds, and back-to-back steps each pay for the write-back of the rows
+    # the previous one left dirty in L2 (a flush by writing a large buffer
+    # would instead charge the step with the flush buffer's write-back).
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    for _ in range(args.warmup):
+        step(g["kv"], g["seq_ids"], g["positions"], stream)
+    torch.cuda.synchronize(dev)
+    K = args.steps
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local, interval_s=0.002)
+    if world > 1:
+        dist.barrier(device_ids=[local])
+    torch.cuda.synchronize(dev)
+    with sampler:
+        e0.record(stream)
+        for i in range(K):
+            step(g["kv"], g["seq_ids"], g["positions"], stream)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier(device_ids=[local])
+    (ms,) = max_over_ranks([e0.elapsed_time(e1) / K], world, dev)
+    if int(err.item()) != 0:
+        raise RuntimeError(f"insert flagged bad tokens: {int(err.item()):#x}")
+
+    # end to end: the new rows, sequence ids and positions copied in from
+    # pinned host memory every step, the error word read back
+    host = {k: d[k].pin_memory() for k in ("kv", "seq_ids", "positions")}
+    dev_in = {k: torch.empty_like(v, device=dev) for k, v in host.items()}
+    host_err = torch.zeros(1, dtype=torch.int32).pin_memory()
+    K2 = max(3, min(K, 50))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    for _ in range(K2):
+        for k, v in host.items():
+            dev_in[k].copy_(v, non_blocking=True)
+        step(dev_in["kv"], dev_in["seq_ids"], dev_in["positions"], stream)
+        host_err.copy_(err, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    (e2e_ms,) = max_over_ranks([e0.elapsed_time(e1) / K2], world, dev)
+
+    peaks, peak_src = load_peaks()
+    gbs = acc["bytes"] / (ms / 1e3) / 1e9
+    line = {
+        "metric": INSERT_METRIC, "value": world * acc["tokens"] / (ms / 1e3), "unit": INSERT_UNIT, "n_gpus": world,
+        "steps": K, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": dict(cfg, l2=f"no flush: {acc['bytes'] / 1e6:.0f} MB moved per step against a {l2 / 1e6:.0f} MB "
+                                f"L2; back-to-back steps, each paying the previous one's write-backs",
+                       parallelism=f"replicas x{world}"),
+        "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": gbs / peaks["hbm_gbs"], "traffic": None, "kernel": "mla_insert_kernel",
+                     "peak_source": peak_src},
+        "e2e": {"value": world * acc["tokens"] / (e2e_ms / 1e3), "unit": INSERT_UNIT,
+                "h2d_bytes_per_step": acc["h2d_bytes"], "d2h_bytes_per_step": acc["d2h_bytes"], "ms_per_step": e2e_ms},
+        "gpu_launches": K,
+        "clocks": sampler.summary(),
+    }
+    if rank == 0 and world == 1:
+        torch.set_num_threads(os.cpu_count() or 1)
+        n, secs = insert_oracle_sample(d, args.cpu_budget)
+        line["cpu_baseline"] = {"value": n / secs, "unit": INSERT_UNIT, "cores": torch.get_num_threads(),
+                                "kind": "oracle",
+                                "sample": f"{n} tokens of sequence 0 (wrapping round), float64, {secs:.1f} s"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
 # ---------------------------------------------------------------- GPU arm
 
 
@@ -261,6 +419,10 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle time for cpu_baseline")
     ap.add_argument("--profile", action="store_true", help="kernel launches only (for ncu): no e2e/oracle/clocks")
     ap.add_argument("--num-sms", type=int, default=0)
+    ap.add_argument("--op", default="decode", choices=["decode", "insert"],
+                    help="decode: the decode step (default); insert: the latent-cache insert alone")
+    ap.add_argument("--insert-batch", type=int, default=64)
+    ap.add_argument("--insert-tokens", type=int, default=1024, help="new tokens per sequence for --op insert")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -269,6 +431,10 @@ def main():
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if args.gpus != world and world > 1:
         args.gpus = world
+
+    if args.op == "insert":
+        run_insert_bench(args, world, rank, local)
+        return
 
     inp = make_inputs(args.workload)
 

@@ -76,6 +76,7 @@ typedef enum {
 #define MLA_DEVERR_PAGE_ID 0x2u /* block_table entry outside [0, num_pages): that page skipped */
 #define MLA_DEVERR_INDEX 0x4u   /* sparse index outside [-1, L_b): that index skipped */
 #define MLA_DEVERR_TIMEOUT 0x8u /* a pipeline wait ran out: results are invalid */
+#define MLA_DEVERR_POSITION 0x10u /* mla_cache_insert: sequence id or position out of range: token skipped */
 
 typedef struct {
   int32_t batch;             /* B >= 0 */
@@ -165,6 +166,56 @@ MLA_API mla_status_t mla_get_error(const void* plan, uint32_t* error_bits, mla_s
 MLA_API mla_status_t mla_decode_noalloc(const mla_decode_desc_t* desc, const int32_t* seq_lens, const void* q,
                                         const void* kv_cache, const int32_t* block_table,
                                         const int32_t* topk_indices, void* out, float* lse, mla_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * Cache insert: the step before decode that fills the paged cache.
+ *
+ * For each new token n (sequence b = seq_ids[n], position p = positions[n]):
+ *
+ *   x      = kv[n, 0:512]   (the latent c_kv)        r = kv[n, 512:576]  (k_pe)
+ *   xn     = bf16( x / sqrt(mean(x^2) + eps) )        (computed in float32)
+ *   row    = kv_cache[block_table[b][p / 64]][p % 64]
+ *   row[0:512]        = bf16( weight * xn )
+ *   row[512 + 2i]     = bf16( r[2i] cos[p][i] - r[2i+1] sin[p][i] )
+ *   row[512 + 2i + 1] = bf16( r[2i] sin[p][i] + r[2i+1] cos[p][i] )   i < 32
+ *
+ * The latent is kv_norm'd and k_pe rotated before they are cached, as in the
+ * absorbed branch of "深度解读DeepSeek：源码解读 DeepSeek-V3", section "MLA";
+ * the RMSNorm's float32 arithmetic, cast and weight order follow
+ * "DeepSeek-V2-Lite 模型结构详解", section "四、RMSNorm". The rotation pairs
+ * consecutive elements; the cos/sin tables (the model's RoPE frequencies,
+ * evaluated at each position) are the caller's.
+ *
+ *   kv          bf16 [N, 576]   (16-byte aligned, dense)
+ *   weight      bf16 [512]      kv_norm weight (16-byte aligned)
+ *   cos_table, sin_table  fp32 [max_positions, 32]
+ *   seq_ids, positions    int32 [N]
+ *   block_table int32 [batch, max_pages_per_seq]
+ *   kv_cache    bf16 [num_pages, 64, 576]   rows are overwritten in place
+ *   error_word  device uint32 or NULL: bits are OR-ed in, never cleared
+ *
+ * A token whose sequence id or position is out of range (b outside
+ * [0, batch), p outside [0, min(max_pages_per_seq * 64, max_positions)))
+ * sets MLA_DEVERR_POSITION, one whose page id is outside [0, num_pages) sets
+ * MLA_DEVERR_PAGE_ID; either is skipped and the others are written. Two
+ * tokens that address the same row race: which one lands is unspecified.
+ * One kernel, asynchronous on `stream`, no allocation. */
+typedef struct {
+  int32_t num_tokens;        /* N >= 0 */
+  int32_t batch;             /* rows of block_table, >= 0 */
+  int32_t max_pages_per_seq; /* block_table row stride (entries), >= 1 */
+  int32_t num_pages;         /* physical pages in kv_cache, >= 1 */
+  int32_t max_positions;     /* rows of cos_table / sin_table, >= 1 */
+  int32_t d_latent;          /* must be 512 */
+  int32_t d_rope;            /* must be 64 */
+  int32_t page_size;         /* must be 64 */
+  float eps;                 /* RMSNorm epsilon, finite, >= 0 */
+} mla_insert_desc_t;
+
+MLA_API mla_status_t mla_cache_insert(const mla_insert_desc_t* desc, const void* kv, const void* weight,
+                                      const float* cos_table, const float* sin_table, const int32_t* seq_ids,
+                                      const int32_t* positions, const int32_t* block_table, void* kv_cache,
+                                      uint32_t* error_word, mla_stream_t stream);
 
 /* Static string for a status code. */
 MLA_API const char* mla_status_string(mla_status_t status);

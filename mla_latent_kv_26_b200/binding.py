@@ -26,10 +26,11 @@ MLA_DEVERR_SEQ_LEN = 0x1
 MLA_DEVERR_PAGE_ID = 0x2
 MLA_DEVERR_INDEX = 0x4
 MLA_DEVERR_TIMEOUT = 0x8
+MLA_DEVERR_POSITION = 0x10
 
 EXPORTED = (
     "mla_plan_bytes", "mla_workspace_bytes", "mla_num_workers", "mla_decode_plan", "mla_decode",
-    "mla_combine", "mla_get_error", "mla_status_string", "mla_decode_noalloc",
+    "mla_combine", "mla_get_error", "mla_status_string", "mla_decode_noalloc", "mla_cache_insert",
 )
 
 DEFAULT_SOFTMAX_SCALE = 1.0 / math.sqrt(192.0)
@@ -59,6 +60,27 @@ def make_desc(*, batch: int, q_len: int, num_heads: int, num_pages: int, max_pag
                              topk, int(bool(causal)), softmax_scale, num_sms)
 
 
+class mla_insert_desc_t(ctypes.Structure):
+    _fields_ = [
+        ("num_tokens", ctypes.c_int32),
+        ("batch", ctypes.c_int32),
+        ("max_pages_per_seq", ctypes.c_int32),
+        ("num_pages", ctypes.c_int32),
+        ("max_positions", ctypes.c_int32),
+        ("d_latent", ctypes.c_int32),
+        ("d_rope", ctypes.c_int32),
+        ("page_size", ctypes.c_int32),
+        ("eps", ctypes.c_float),
+    ]
+
+
+def make_insert_desc(*, num_tokens: int, batch: int, max_pages_per_seq: int, num_pages: int, max_positions: int,
+                     eps: float = 1e-6, d_latent: int = 512, d_rope: int = 64,
+                     page_size: int = 64) -> mla_insert_desc_t:
+    return mla_insert_desc_t(num_tokens, batch, max_pages_per_seq, num_pages, max_positions, d_latent, d_rope,
+                             page_size, eps)
+
+
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
         raise RuntimeError(
@@ -77,6 +99,7 @@ def _load() -> ctypes.CDLL:
         "mla_get_error": (ctypes.c_int, [P, ctypes.POINTER(ctypes.c_uint32), P]),
         "mla_status_string": (ctypes.c_char_p, [ctypes.c_int]),
         "mla_decode_noalloc": (ctypes.c_int, [D, P, P, P, P, P, P, P, P]),
+        "mla_cache_insert": (ctypes.c_int, [ctypes.POINTER(mla_insert_desc_t), P, P, P, P, P, P, P, P, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -147,6 +170,14 @@ def mla_decode_noalloc(desc, seq_lens, q, kv_cache, block_table, topk_indices, o
     """Plan + decode + combine with the library's fixed device scratch (no allocation)."""
     return int(_lib.mla_decode_noalloc(ctypes.byref(desc), _ptr(seq_lens), _ptr(q), _ptr(kv_cache), _ptr(block_table),
                                        _ptr(topk_indices), _ptr(out), _ptr(lse), _stream(stream)))
+
+
+def mla_cache_insert(desc, kv, weight, cos_table, sin_table, seq_ids, positions, block_table, kv_cache,
+                     error_word=None, stream=None) -> int:
+    """kv_norm + RoPE of new tokens, written into their rows of the paged cache."""
+    return int(_lib.mla_cache_insert(ctypes.byref(desc), _ptr(kv), _ptr(weight), _ptr(cos_table), _ptr(sin_table),
+                                     _ptr(seq_ids), _ptr(positions), _ptr(block_table), _ptr(kv_cache),
+                                     _ptr(error_word), _stream(stream)))
 
 
 def mla_get_error(plan, stream=None):

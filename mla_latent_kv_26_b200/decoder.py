@@ -83,3 +83,33 @@ def decoder_for(inputs: dict, *, num_sms: int = 0, device="cuda", **kw) -> MlaDe
     return MlaDecoder(batch=inputs["batch"], q_len=inputs["q_len"], num_heads=inputs["heads"],
                       num_pages=inputs["num_pages"], max_pages_per_seq=inputs["max_pages_per_seq"],
                       topk=inputs["topk"], causal=inputs["causal"], num_sms=num_sms, device=device, **kw)
+
+
+def cache_insert(kv: torch.Tensor, weight: torch.Tensor, cos: torch.Tensor, sin: torch.Tensor, seq_ids: torch.Tensor,
+                 positions: torch.Tensor, block_table: torch.Tensor, kv_cache: torch.Tensor, *, eps: float = 1e-6,
+                 error_word: Optional[torch.Tensor] = None, stream=None) -> None:
+    """kv_norm + RoPE of the new tokens' rows ``kv`` [N, 576], written in place
+    into their rows of ``kv_cache`` [pages, 64, 576] (one library kernel).
+    ``error_word``: optional int32 [1] device tensor that collects the
+    MLA_DEVERR bits of skipped tokens."""
+    dev = kv_cache.device
+    n = kv.shape[0] if kv.dim() == 2 else -1
+    want = [("kv", kv, torch.bfloat16, (n, 576)), ("weight", weight, torch.bfloat16, (512,)),
+            ("cos", cos, torch.float32, (cos.shape[0], 32)), ("sin", sin, torch.float32, tuple(cos.shape)),
+            ("seq_ids", seq_ids, torch.int32, (n,)), ("positions", positions, torch.int32, (n,)),
+            ("block_table", block_table, torch.int32, None), ("kv_cache", kv_cache, torch.bfloat16, None)]
+    for name, t, dtype, shape in want:
+        if t.device != dev or t.dtype != dtype or not t.is_contiguous():
+            raise ValueError(f"{name}: need a contiguous {dtype} tensor on {dev}")
+        if shape is not None and tuple(t.shape) != tuple(shape):
+            raise ValueError(f"{name}: shape {tuple(t.shape)} != {tuple(shape)}")
+    if block_table.dim() != 2 or kv_cache.dim() != 3 or tuple(kv_cache.shape[1:]) != (64, 576):
+        raise ValueError("block_table must be [batch, max_pages_per_seq], kv_cache [pages, 64, 576]")
+    if error_word is not None and (error_word.device != dev or error_word.dtype != torch.int32):
+        raise ValueError("error_word: need an int32 tensor on the cache's device")
+    desc = B.make_insert_desc(num_tokens=n, batch=block_table.shape[0], max_pages_per_seq=max(block_table.shape[1], 1),
+                              num_pages=kv_cache.shape[0], max_positions=cos.shape[0], eps=eps)
+    s = torch.cuda.current_stream(dev) if stream is None else stream
+    with torch.cuda.device(dev):
+        B.check(B.mla_cache_insert(desc, kv, weight, cos, sin, seq_ids, positions, block_table, kv_cache, error_word,
+                                   s), "mla_cache_insert")

@@ -154,3 +154,42 @@ def small(key: str = "t", *, batch: int, heads: int, q_len: int = 1, lens: Seque
                  causal=causal, q_std=q_std, cache_std=cache_std, seed=seed)
     return make_inputs(w, lens=lens, **kw)
 
+
+
+def insert_inputs(*, lens: Sequence[int], new_tokens: Sequence[int], seed: int = 0, kv_std: float = 1.0,
+                  rope_base: float = 10000.0, slack_pages: int = 2) -> dict:
+    """Inputs of a latent-cache insert: sequence b already holds
+    ``lens[b] - new_tokens[b]`` tokens and appends ``new_tokens[b]`` more at
+    positions ``lens[b] - new_tokens[b] .. lens[b] - 1`` (a prefill chunk when
+    that is the whole sequence, one decode token when it is 1).
+
+    Draw order, from one generator: page permutation -> prior cache contents ->
+    new rows ``kv`` [N, 576] (N(0, kv_std)) -> kv_norm weight (N(1, 0.1^2)).
+    ``cos``/``sin`` [max(lens), 32] are the RoPE tables of the caller at angle
+    ``pos * rope_base ** (-i / 32)`` for pair i (the usual RoPE frequency
+    ladder; the method takes any table)."""
+    g = torch.Generator().manual_seed(seed)
+    lens = [int(x) for x in lens]
+    new_tokens = [int(x) for x in new_tokens]
+    npg = [max((L + PAGE - 1) // PAGE, 1) for L in lens]
+    maxp = max(npg) if npg else 1
+    num_pages = sum(npg) + slack_pages
+    perm = torch.randperm(num_pages, generator=g).to(torch.int32)
+    bt = torch.full((len(lens), maxp), -1, dtype=torch.int32)
+    k = 0
+    for b, n in enumerate(npg):
+        bt[b, :n] = perm[k:k + n]
+        k += n
+    cache = torch.randn(num_pages, PAGE, D_QK, generator=g).to(torch.bfloat16)
+    seq_ids = torch.cat([torch.full((n,), b, dtype=torch.int32) for b, n in enumerate(new_tokens)])
+    positions = torch.cat([torch.arange(L - n, L, dtype=torch.int32) for L, n in zip(lens, new_tokens)])
+    kv = (torch.randn(len(seq_ids), D_QK, generator=g) * kv_std).to(torch.bfloat16)
+    weight = (1.0 + 0.1 * torch.randn(D_LATENT, generator=g)).to(torch.bfloat16)
+    max_pos = max(lens) if lens else 1
+    inv_freq = rope_base ** (-torch.arange(32, dtype=torch.float64) / 32.0)
+    ang = torch.arange(max_pos, dtype=torch.float64)[:, None] * inv_freq[None, :]
+    return {
+        "kv": kv, "weight": weight, "cos": torch.cos(ang).float(), "sin": torch.sin(ang).float(),
+        "seq_ids": seq_ids, "positions": positions, "block_table": bt, "cache": cache,
+        "batch": len(lens), "num_pages": num_pages, "max_pages_per_seq": maxp, "lens": lens,
+    }

@@ -24,8 +24,8 @@ def _declared():
 
 def test_header_declares_the_boundary():
     assert _declared() == sorted([
-        "mla_combine", "mla_decode", "mla_decode_noalloc", "mla_decode_plan", "mla_get_error", "mla_num_workers",
-        "mla_plan_bytes", "mla_status_string", "mla_workspace_bytes"])
+        "mla_cache_insert", "mla_combine", "mla_decode", "mla_decode_noalloc", "mla_decode_plan", "mla_get_error",
+        "mla_num_workers", "mla_plan_bytes", "mla_status_string", "mla_workspace_bytes"])
 
 
 def test_library_exports_every_declared_symbol(libmla):
@@ -87,6 +87,38 @@ def test_null_and_misaligned_pointers_rejected(libmla):
     assert libmla.mla_combine(d, 16, 16, 1 << 30, 16, 18, None) == INV       # lse not 4-B aligned
     st, _ = libmla.mla_get_error(None)
     assert st == INV
+
+
+def _idesc(libmla, **kw):
+    base = dict(num_tokens=4, batch=2, max_pages_per_seq=4, num_pages=8, max_positions=256)
+    base.update(kw)
+    return libmla.make_insert_desc(**base)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(num_tokens=-1), 1), (dict(batch=-1), 1), (dict(max_pages_per_seq=0), 1), (dict(num_pages=0), 1),
+    (dict(max_positions=0), 1), (dict(eps=-1e-6), 1), (dict(eps=float("nan")), 1), (dict(eps=float("inf")), 1),
+    (dict(d_latent=256), 2), (dict(d_rope=32), 2), (dict(page_size=16), 2),
+])
+def test_cache_insert_bad_descriptors_rejected(libmla, kw, status):
+    d = _idesc(libmla, **kw)
+    assert libmla.mla_cache_insert(d, 16, 16, 16, 16, 16, 16, 16, 16, None, None) == status
+
+
+def test_cache_insert_null_misaligned_and_empty(libmla):
+    d = _idesc(libmla)
+    good = [16, 16, 16, 16, 16, 16, 16, 16]
+    for i in range(8):
+        args = list(good)
+        args[i] = None
+        assert libmla.mla_cache_insert(d, *args, None, None) == libmla.MLA_ERR_INVALID_ARG, i
+    for i, off in ((0, 8), (1, 8), (2, 2), (3, 2), (7, 8)):
+        args = list(good)
+        args[i] += off
+        assert libmla.mla_cache_insert(d, *args, None, None) == libmla.MLA_ERR_INVALID_ARG, i
+    assert libmla.mla_cache_insert(d, *good, 18, None) == libmla.MLA_ERR_INVALID_ARG
+    # no tokens: nothing to do, no pointer is read and nothing is launched
+    assert libmla.mla_cache_insert(_idesc(libmla, num_tokens=0), *([None] * 8), None, None) == libmla.MLA_OK
 
 
 def test_plan_too_small_rejected(libmla):
