@@ -82,25 +82,29 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def decode_source_sha() -> str:
+DECODE_SOURCES = ("mla_decode.cu", "sm100.cuh", "common.cuh")
+INSERT_SOURCES = ("mla_insert.cu", "sm100.cuh", "common.cuh")
+
+
+def decode_source_sha(files=DECODE_SOURCES) -> str:
     h = hashlib.sha256()
-    for f in ("mla_decode.cu", "sm100.cuh", "common.cuh"):
+    for f in files:
         with open(os.path.join(ROOT, "mla_latent_kv_26_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(workload: str):
-    """DRAM bytes per decode launch from the committed ncu summary, if it was
-    taken on the current kernel source; else None."""
-    path = os.path.join(ROOT, "profiles", f"mla_decode_kernel_{workload}.md")
+def profiled_traffic(workload: str, kernel: str = "mla_decode_kernel", files=DECODE_SOURCES):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel source; else None."""
+    path = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.md")
     try:
         text = open(path).read()
     except OSError:
         return None
     m_sha = re.search(r"source_sha:\s*([0-9a-f]+)", text)
     m_b = re.search(r"dram_bytes_per_launch:\s*([0-9]+)", text)
-    if not m_sha or not m_b or m_sha.group(1) != decode_source_sha():
+    if not m_sha or not m_b or m_sha.group(1) != decode_source_sha(files):
         return None
     return int(m_b.group(1))
 
@@ -387,7 +391,8 @@ def run_insert_bench(args, world, rank, local):
                                 f"L2; back-to-back steps, each paying the previous one's write-backs",
                        parallelism=f"replicas x{world}"),
         "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                     "frac": gbs / peaks["hbm_gbs"], "traffic": None, "kernel": "mla_insert_kernel",
+                     "frac": gbs / peaks["hbm_gbs"], "kernel": "mla_insert_kernel",
+                     "traffic": profiled_traffic(f"prefill{B}x{T}", "mla_insert_kernel", INSERT_SOURCES),
                      "peak_source": peak_src},
         "e2e": {"value": world * acc["tokens"] / (e2e_ms / 1e3), "unit": INSERT_UNIT,
                 "h2d_bytes_per_step": acc["h2d_bytes"], "d2h_bytes_per_step": acc["d2h_bytes"], "ms_per_step": e2e_ms},

@@ -27,7 +27,6 @@ __host__ __device__ inline int plan_ntok_off(int tasks) { return kPlanHeader + t
 __host__ __device__ inline int plan_words(int tasks) { return kPlanHeader + 2 * tasks + 1; }
 
 constexpr uint32_t kErrSeqLen = 0x1u, kErrPageId = 0x2u, kErrIndex = 0x4u, kErrTimeout = 0x8u;
-constexpr uint32_t kErrInsertPos = 0x10u;  // cache insert: sequence id or position out of range
 
 struct PlanArgs {
   const int32_t* seq_lens;

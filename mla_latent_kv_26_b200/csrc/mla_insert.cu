@@ -45,6 +45,10 @@ struct InsertArgs {
 
 namespace {
 
+// Device error bit of a token whose sequence id or position is out of range
+// (MLA_DEVERR_POSITION; the other bits are shared with decode).
+constexpr uint32_t kErrInsertPos = 0x10u;
+
 #ifndef MLA_INSERT_UNROLL
 #define MLA_INSERT_UNROLL 1
 #endif
