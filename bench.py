@@ -411,6 +411,166 @@ def run_insert_bench(args, world, rank, local):
         dist.destroy_process_group()
 
 
+# ---------------------------------------------------------------- absorb / un-absorb (--op absorb)
+
+ABSORB_METRIC = "MLA absorb + un-absorb projection tokens/s (W_UK^T q_nope, W_UV o_lat) and achieved GB/s vs HBM roofline"
+
+
+def absorb_accounting(T: int, H: int) -> dict:
+    """Algorithmic bytes of one absorb + un-absorb pass: both weight halves
+    once, q [T,H,192] and q_abs [T,H,576] (absorb), o_lat [T,H,512] and out
+    [T,H,128] (un-absorb)."""
+    w = H * 128 * 512 * 2
+    absorb = w + T * H * (192 + 576) * 2
+    unabsorb = w + T * H * (512 + 128) * 2
+    flops = 2 * T * H * 128 * 512 * 2
+    return {"absorb": absorb, "unabsorb": unabsorb, "bytes": absorb + unabsorb, "flops": flops,
+            "h2d_bytes": T * H * (192 + 512) * 2, "d2h_bytes": T * H * (576 + 128) * 2}
+
+
+def absorb_oracle_sample(d: dict, budget_s: float):
+    import oracle
+
+    t0, done = time.perf_counter(), 0
+    w_uk, w_uv = d["wkv_b"][:, :128, :], d["wkv_b"][:, 128:, :]
+    while time.perf_counter() - t0 < budget_s:
+        t = done % d["tokens"]
+        oracle.absorb_query(d["q"][t, :, :128], w_uk)
+        oracle.unabsorb_output(d["o_lat"][t], w_uv)
+        done += 1
+    return done, time.perf_counter() - t0
+
+
+def run_absorb_bench(args, world, rank, local):
+    from mla_latent_kv_26_b200.workloads import absorb_inputs
+
+    T, H = args.absorb_tokens, 128
+    d = absorb_inputs(tokens=T, heads=H, seed=6)
+    acc = absorb_accounting(T, H)
+    cfg = {"workload": f"absorb-t{T}-h{H}: {T} decode tokens x {H} heads, wkv_b [H,256,512] bf16",
+           "tokens_per_step": T, "bytes_per_step": acc["bytes"], "flops_per_step": acc["flops"]}
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        torch.set_num_threads(os.cpu_count() or 1)
+        toks, secs = 0, 0.0
+        for s in range(args.warmup + args.steps):
+            n, dt = absorb_oracle_sample(d, 0.2)
+            if s >= args.warmup:
+                toks, secs = toks + n, secs + dt
+        v = toks / secs
+        print(json.dumps({
+            "impl": "reference", "metric": ABSORB_METRIC, "value": v, "unit": INSERT_UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": cfg,
+            "cpu_baseline": {"value": v, "unit": INSERT_UNIT, "cores": torch.get_num_threads(), "kind": "oracle",
+                             "sample": "float64 oracle projections, about 0.2 s of tokens per step"},
+            "e2e": {"value": v, "unit": INSERT_UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}), flush=True)
+        return
+
+    import torch.distributed as dist
+
+    from mla_latent_kv_26_b200.decoder import absorb_query, unabsorb_output
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+    g = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in d.items()}
+    q_abs = torch.empty(T, H, 576, dtype=torch.bfloat16, device=dev)
+    out = torch.empty(T, H, 128, dtype=torch.bfloat16, device=dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    # The weights (33.5 MB) fit in L2: before every timed step the L2 is
+    # flushed by READING a buffer twice its size, which leaves it full of clean
+    # lines (a flush by writing would charge the step with the write-back of
+    # the flush buffer's dirty lines).
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush_buf = torch.ones(2 * l2 // 4, dtype=torch.float32, device=dev)
+    sink = torch.empty(1, dtype=torch.float32, device=dev)
+    for _ in range(args.warmup):
+        absorb_query(g["q"], g["wkv_b"], q_abs, error_word=err)
+        unabsorb_output(g["o_lat"], g["wkv_b"], out, error_word=err)
+    torch.cuda.synchronize(dev)
+    K = args.steps
+    ev = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(3)) for _ in range(K)]
+    sampler = ClockSampler(local, interval_s=0.002)
+    if world > 1:
+        dist.barrier(device_ids=[local])
+    torch.cuda.synchronize(dev)
+    with sampler:
+        for i in range(K):
+            torch.sum(flush_buf, dim=0, out=sink)
+            ev[i][0].record(stream)
+            absorb_query(g["q"], g["wkv_b"], q_abs, error_word=err)
+            ev[i][1].record(stream)
+            unabsorb_output(g["o_lat"], g["wkv_b"], out, error_word=err)
+            ev[i][2].record(stream)
+        torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier(device_ids=[local])
+    a_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / K
+    u_ms = sum(e[1].elapsed_time(e[2]) for e in ev) / K
+    ms = sum(e[0].elapsed_time(e[2]) for e in ev) / K
+    ms, a_ms, u_ms = max_over_ranks([ms, a_ms, u_ms], world, dev)
+    if int(err.item()) != 0:
+        raise RuntimeError(f"device error word {int(err.item()):#x}")
+
+    # end to end: q and o_lat from pinned host memory, q_abs and out back, every step
+    hq, ho = d["q"].pin_memory(), d["o_lat"].pin_memory()
+    hqa = torch.empty(T, H, 576, dtype=torch.bfloat16).pin_memory()
+    hout = torch.empty(T, H, 128, dtype=torch.bfloat16).pin_memory()
+    dq, do = torch.empty_like(g["q"]), torch.empty_like(g["o_lat"])
+    K2 = max(3, min(K, 50))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    for _ in range(K2):
+        dq.copy_(hq, non_blocking=True)
+        do.copy_(ho, non_blocking=True)
+        absorb_query(dq, g["wkv_b"], q_abs, error_word=err)
+        unabsorb_output(do, g["wkv_b"], out, error_word=err)
+        hqa.copy_(q_abs, non_blocking=True)
+        hout.copy_(out, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    (e2e_ms,) = max_over_ranks([e0.elapsed_time(e1) / K2], world, dev)
+
+    peaks, peak_src = load_peaks()
+    gbs = acc["bytes"] / (ms / 1e3) / 1e9
+    a_gbs = acc["absorb"] / (a_ms / 1e3) / 1e9
+    u_gbs = acc["unabsorb"] / (u_ms / 1e3) / 1e9
+    line = {
+        "metric": ABSORB_METRIC, "value": world * T / (ms / 1e3), "unit": INSERT_UNIT, "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic",
+        "config": dict(cfg, l2=f"L2 flushed before every timed step by reading a {2 * l2 / 1e6:.0f} MB buffer",
+                       parallelism=f"replicas x{world}"),
+        "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": gbs / peaks["hbm_gbs"], "traffic": None,
+                     "kernel": "mla_absorb_q_kernel + mla_unabsorb_o_kernel", "peak_source": peak_src,
+                     "absorb_us": a_ms * 1e3, "absorb_frac": a_gbs / peaks["hbm_gbs"],
+                     "unabsorb_us": u_ms * 1e3, "unabsorb_frac": u_gbs / peaks["hbm_gbs"],
+                     "tflop_per_s": acc["flops"] / (ms / 1e3) / 1e12},
+        "e2e": {"value": world * T / (e2e_ms / 1e3), "unit": INSERT_UNIT, "h2d_bytes_per_step": acc["h2d_bytes"],
+                "d2h_bytes_per_step": acc["d2h_bytes"], "ms_per_step": e2e_ms},
+        "gpu_launches": 2 * K,
+        "clocks": sampler.summary(),
+    }
+    if rank == 0 and world == 1:
+        torch.set_num_threads(os.cpu_count() or 1)
+        n, secs = absorb_oracle_sample(d, args.cpu_budget)
+        line["cpu_baseline"] = {"value": n / secs, "unit": INSERT_UNIT, "cores": torch.get_num_threads(),
+                                "kind": "oracle", "sample": f"{n} tokens (absorb + un-absorb), float64, {secs:.1f} s"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
 # ---------------------------------------------------------------- GPU arm
 
 
@@ -424,8 +584,10 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle time for cpu_baseline")
     ap.add_argument("--profile", action="store_true", help="kernel launches only (for ncu): no e2e/oracle/clocks")
     ap.add_argument("--num-sms", type=int, default=0)
-    ap.add_argument("--op", default="decode", choices=["decode", "insert"],
-                    help="decode: the decode step (default); insert: the latent-cache insert alone")
+    ap.add_argument("--op", default="decode", choices=["decode", "insert", "absorb"],
+                    help="decode: the decode step (default); insert: the latent-cache insert alone; "
+                         "absorb: the absorb + un-absorb projections")
+    ap.add_argument("--absorb-tokens", type=int, default=64, help="query tokens for --op absorb")
     ap.add_argument("--insert-batch", type=int, default=64)
     ap.add_argument("--insert-tokens", type=int, default=1024, help="new tokens per sequence for --op insert")
     args = ap.parse_args()
@@ -439,6 +601,9 @@ def main():
 
     if args.op == "insert":
         run_insert_bench(args, world, rank, local)
+        return
+    if args.op == "absorb":
+        run_absorb_bench(args, world, rank, local)
         return
 
     inp = make_inputs(args.workload)

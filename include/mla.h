@@ -217,6 +217,42 @@ MLA_API mla_status_t mla_cache_insert(const mla_insert_desc_t* desc, const void*
                                       const int32_t* positions, const int32_t* block_table, void* kv_cache,
                                       uint32_t* error_word, mla_stream_t stream);
 
+/* ---------------------------------------------------------------------------
+ * Absorb / un-absorb: the per-head projections around the latent decode.
+ *
+ * wkv_b is the model's kv up-projection viewed as [H, 256, 512] bf16: rows
+ * [0, 128) of head h are W_UK[h] and rows [128, 256) are W_UV[h]
+ * ("深度解读DeepSeek：源码解读 DeepSeek-V3", section "MLA", absorbed branch;
+ * "DeepSeek-V2-Lite 模型结构详解", section "五、MLA：注意力", the two absorption
+ * identities). For T tokens (T = B * Sq of a decode step):
+ *
+ *   mla_absorb_query:    q_abs[t, h, 0:512]   = sum_d q[t, h, d] * W_UK[h][d, 0:512]   (d < 128)
+ *                        q_abs[t, h, 512:576] = q[t, h, 128:192]                       (q_pe, copied)
+ *   mla_unabsorb_output: out[t, h, v]         = sum_c W_UV[h][v, c] * o_lat[t, h, c]   (v < 128, c < 512)
+ *
+ * so that q_abs is mla_decode's query and o_lat its latent output. bf16 in
+ * and out, fp32 accumulation on the tensor cores, one kernel each.
+ *
+ *   q      bf16 [T, H, 192]  (q_nope[128] || q_pe[64], as the q projection emits it)
+ *   q_abs  bf16 [T, H, 576]  o_lat bf16 [T, H, 512]  out bf16 [T, H, 128]
+ *   wkv_b  bf16 [H, 256, 512]
+ * All pointers 16-byte aligned, densely packed; error_word: device uint32 or
+ * NULL, MLA_DEVERR_TIMEOUT is OR-ed in if a bounded device wait ran out
+ * (results then invalid). Asynchronous on `stream`, no allocation. */
+typedef struct {
+  int32_t num_tokens; /* T >= 0 */
+  int32_t num_heads;  /* H: 1..128 */
+  int32_t d_nope;     /* must be 128 (qk_nope_head_dim) */
+  int32_t d_rope;     /* must be 64 (qk_rope_head_dim) */
+  int32_t d_latent;   /* must be 512 (kv_lora_rank) */
+  int32_t d_v;        /* must be 128 (v_head_dim) */
+} mla_absorb_desc_t;
+
+MLA_API mla_status_t mla_absorb_query(const mla_absorb_desc_t* desc, const void* q, const void* wkv_b, void* q_abs,
+                                      uint32_t* error_word, mla_stream_t stream);
+MLA_API mla_status_t mla_unabsorb_output(const mla_absorb_desc_t* desc, const void* o_lat, const void* wkv_b,
+                                         void* out, uint32_t* error_word, mla_stream_t stream);
+
 /* Static string for a status code. */
 MLA_API const char* mla_status_string(mla_status_t status);
 

@@ -31,6 +31,7 @@ MLA_DEVERR_POSITION = 0x10
 EXPORTED = (
     "mla_plan_bytes", "mla_workspace_bytes", "mla_num_workers", "mla_decode_plan", "mla_decode",
     "mla_combine", "mla_get_error", "mla_status_string", "mla_decode_noalloc", "mla_cache_insert",
+    "mla_absorb_query", "mla_unabsorb_output",
 )
 
 DEFAULT_SOFTMAX_SCALE = 1.0 / math.sqrt(192.0)
@@ -81,6 +82,22 @@ def make_insert_desc(*, num_tokens: int, batch: int, max_pages_per_seq: int, num
                              page_size, eps)
 
 
+class mla_absorb_desc_t(ctypes.Structure):
+    _fields_ = [
+        ("num_tokens", ctypes.c_int32),
+        ("num_heads", ctypes.c_int32),
+        ("d_nope", ctypes.c_int32),
+        ("d_rope", ctypes.c_int32),
+        ("d_latent", ctypes.c_int32),
+        ("d_v", ctypes.c_int32),
+    ]
+
+
+def make_absorb_desc(*, num_tokens: int, num_heads: int, d_nope: int = 128, d_rope: int = 64, d_latent: int = 512,
+                     d_v: int = 128) -> mla_absorb_desc_t:
+    return mla_absorb_desc_t(num_tokens, num_heads, d_nope, d_rope, d_latent, d_v)
+
+
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
         raise RuntimeError(
@@ -100,6 +117,8 @@ def _load() -> ctypes.CDLL:
         "mla_status_string": (ctypes.c_char_p, [ctypes.c_int]),
         "mla_decode_noalloc": (ctypes.c_int, [D, P, P, P, P, P, P, P, P]),
         "mla_cache_insert": (ctypes.c_int, [ctypes.POINTER(mla_insert_desc_t), P, P, P, P, P, P, P, P, P, P]),
+        "mla_absorb_query": (ctypes.c_int, [ctypes.POINTER(mla_absorb_desc_t), P, P, P, P, P]),
+        "mla_unabsorb_output": (ctypes.c_int, [ctypes.POINTER(mla_absorb_desc_t), P, P, P, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -178,6 +197,18 @@ def mla_cache_insert(desc, kv, weight, cos_table, sin_table, seq_ids, positions,
     return int(_lib.mla_cache_insert(ctypes.byref(desc), _ptr(kv), _ptr(weight), _ptr(cos_table), _ptr(sin_table),
                                      _ptr(seq_ids), _ptr(positions), _ptr(block_table), _ptr(kv_cache),
                                      _ptr(error_word), _stream(stream)))
+
+
+def mla_absorb_query(desc, q, wkv_b, q_abs, error_word=None, stream=None) -> int:
+    """q [T,H,192] -> q_abs [T,H,576] = (W_UK^T q_nope || q_pe)."""
+    return int(_lib.mla_absorb_query(ctypes.byref(desc), _ptr(q), _ptr(wkv_b), _ptr(q_abs), _ptr(error_word),
+                                     _stream(stream)))
+
+
+def mla_unabsorb_output(desc, o_lat, wkv_b, out, error_word=None, stream=None) -> int:
+    """o_lat [T,H,512] -> out [T,H,128] = W_UV o_lat."""
+    return int(_lib.mla_unabsorb_output(ctypes.byref(desc), _ptr(o_lat), _ptr(wkv_b), _ptr(out), _ptr(error_word),
+                                        _stream(stream)))
 
 
 def mla_get_error(plan, stream=None):

@@ -114,6 +114,10 @@ size_t workspace_bytes_for(const mla_decode_desc_t* d, int workers) {
 bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 
 }  // namespace
+
+// The driver's tensor-map encoder, shared with the other entry points.
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() { return encoder(); }
+
 }  // namespace mla
 
 using namespace mla;

@@ -113,3 +113,46 @@ def cache_insert(kv: torch.Tensor, weight: torch.Tensor, cos: torch.Tensor, sin:
     with torch.cuda.device(dev):
         B.check(B.mla_cache_insert(desc, kv, weight, cos, sin, seq_ids, positions, block_table, kv_cache, error_word,
                                    s), "mla_cache_insert")
+
+
+def _check_tensor(name, t, dtype, shape, dev):
+    if t.device != dev or t.dtype != dtype or not t.is_contiguous():
+        raise ValueError(f"{name}: need a contiguous {dtype} tensor on {dev}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: shape {tuple(t.shape)} != {tuple(shape)}")
+
+
+def absorb_query(q: torch.Tensor, wkv_b: torch.Tensor, out: Optional[torch.Tensor] = None, *,
+                 error_word: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """q [T, H, 192] (q_nope || q_pe) and wkv_b [H, 256, 512] -> the decode
+    query [T, H, 576] = (W_UK^T q_nope || q_pe), one library kernel."""
+    T, H = q.shape[0], q.shape[1]
+    dev = q.device
+    _check_tensor("q", q, torch.bfloat16, (T, H, 192), dev)
+    _check_tensor("wkv_b", wkv_b, torch.bfloat16, (H, 256, 512), dev)
+    if out is None:
+        out = torch.empty(T, H, 576, dtype=torch.bfloat16, device=dev)
+    _check_tensor("out", out, torch.bfloat16, (T, H, 576), dev)
+    s = torch.cuda.current_stream(dev) if stream is None else stream
+    with torch.cuda.device(dev):
+        B.check(B.mla_absorb_query(B.make_absorb_desc(num_tokens=T, num_heads=H), q, wkv_b, out, error_word, s),
+                "mla_absorb_query")
+    return out
+
+
+def unabsorb_output(o_lat: torch.Tensor, wkv_b: torch.Tensor, out: Optional[torch.Tensor] = None, *,
+                    error_word: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """o_lat [T, H, 512] (the decode output) and wkv_b [H, 256, 512] -> the
+    per-head values [T, H, 128] = W_UV o_lat, one library kernel."""
+    T, H = o_lat.shape[0], o_lat.shape[1]
+    dev = o_lat.device
+    _check_tensor("o_lat", o_lat, torch.bfloat16, (T, H, 512), dev)
+    _check_tensor("wkv_b", wkv_b, torch.bfloat16, (H, 256, 512), dev)
+    if out is None:
+        out = torch.empty(T, H, 128, dtype=torch.bfloat16, device=dev)
+    _check_tensor("out", out, torch.bfloat16, (T, H, 128), dev)
+    s = torch.cuda.current_stream(dev) if stream is None else stream
+    with torch.cuda.device(dev):
+        B.check(B.mla_unabsorb_output(B.make_absorb_desc(num_tokens=T, num_heads=H), o_lat, wkv_b, out, error_word,
+                                      s), "mla_unabsorb_output")
+    return out

@@ -193,3 +193,16 @@ def insert_inputs(*, lens: Sequence[int], new_tokens: Sequence[int], seed: int =
         "seq_ids": seq_ids, "positions": positions, "block_table": bt, "cache": cache,
         "batch": len(lens), "num_pages": num_pages, "max_pages_per_seq": maxp, "lens": lens,
     }
+
+
+def absorb_inputs(*, tokens: int, heads: int, seed: int = 0, w_std: float = 0.05, o_std: float = 0.3) -> dict:
+    """Inputs of the absorb / un-absorb projections for T = ``tokens`` query
+    tokens: q [T, H, 192] ~ N(0, 1) (q_nope || q_pe), wkv_b [H, 256, 512] ~
+    N(0, w_std^2) (rows 0-127 of a head: W_UK, 128-255: W_UV, as the model's
+    kv up-projection viewed per head), o_lat [T, H, 512] ~ N(0, o_std^2).
+    Draw order: q -> wkv_b -> o_lat."""
+    g = torch.Generator().manual_seed(seed)
+    q = torch.randn(tokens, heads, 192, generator=g).to(torch.bfloat16)
+    wkv_b = (torch.randn(heads, 256, 512, generator=g) * w_std).to(torch.bfloat16)
+    o_lat = (torch.randn(tokens, heads, 512, generator=g) * o_std).to(torch.bfloat16)
+    return {"q": q, "wkv_b": wkv_b, "o_lat": o_lat, "tokens": tokens, "heads": heads}

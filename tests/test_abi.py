@@ -24,8 +24,9 @@ def _declared():
 
 def test_header_declares_the_boundary():
     assert _declared() == sorted([
-        "mla_cache_insert", "mla_combine", "mla_decode", "mla_decode_noalloc", "mla_decode_plan", "mla_get_error",
-        "mla_num_workers", "mla_plan_bytes", "mla_status_string", "mla_workspace_bytes"])
+        "mla_absorb_query", "mla_cache_insert", "mla_combine", "mla_decode", "mla_decode_noalloc", "mla_decode_plan",
+        "mla_get_error", "mla_num_workers", "mla_plan_bytes", "mla_status_string", "mla_unabsorb_output",
+        "mla_workspace_bytes"])
 
 
 def test_library_exports_every_declared_symbol(libmla):
@@ -119,6 +120,32 @@ def test_cache_insert_null_misaligned_and_empty(libmla):
     assert libmla.mla_cache_insert(d, *good, 18, None) == libmla.MLA_ERR_INVALID_ARG
     # no tokens: nothing to do, no pointer is read and nothing is launched
     assert libmla.mla_cache_insert(_idesc(libmla, num_tokens=0), *([None] * 8), None, None) == libmla.MLA_OK
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(num_tokens=-1), 1), (dict(num_heads=0), 1), (dict(num_heads=129), 2), (dict(d_nope=64), 2),
+    (dict(d_rope=32), 2), (dict(d_latent=256), 2), (dict(d_v=64), 2), (dict(num_tokens=65535 * 128 + 1), 2),
+])
+def test_absorb_bad_descriptors_rejected(libmla, kw, status):
+    base = dict(num_tokens=4, num_heads=8)
+    base.update(kw)
+    d = libmla.make_absorb_desc(**base)
+    assert libmla.mla_absorb_query(d, 16, 16, 16, None, None) == status
+    assert libmla.mla_unabsorb_output(d, 16, 16, 16, None, None) == status
+
+
+def test_absorb_null_misaligned_and_empty(libmla):
+    d = libmla.make_absorb_desc(num_tokens=4, num_heads=8)
+    for fn in (libmla.mla_absorb_query, libmla.mla_unabsorb_output):
+        for i in range(3):
+            args = [16, 16, 16]
+            args[i] = None
+            assert fn(d, *args, None, None) == libmla.MLA_ERR_INVALID_ARG, i
+            args = [16, 16, 16]
+            args[i] = 24
+            assert fn(d, *args, None, None) == libmla.MLA_ERR_INVALID_ARG, i
+        assert fn(d, 16, 16, 16, 18, None) == libmla.MLA_ERR_INVALID_ARG
+        assert fn(libmla.make_absorb_desc(num_tokens=0, num_heads=8), None, None, None, None, None) == libmla.MLA_OK
 
 
 def test_plan_too_small_rejected(libmla):
