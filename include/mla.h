@@ -147,7 +147,7 @@ MLA_API mla_status_t mla_get_error(const void* plan, uint32_t* error_bits, mla_s
  * cudaMalloc, for example code running where a caching allocator owns all
  * device memory, or an embedding that forbids allocation while serving.
  * The caller passes inputs and outputs as for mla_decode_plan / mla_decode.
- * The paper has no counterpart; this is an interface convenience.
+ * No source page describes it; this is an interface convenience.
  *
  * - The first call on a device sets up the scratch's device address and the
  *   kernel attributes (with that device current); make that first call before
