@@ -85,3 +85,42 @@ def test_reference_arm_under_torchrun_two_ranks():
     assert line["impl"] == "reference" and line["n_gpus"] == 2
     assert line["value"] > 0 and line["e2e"]["value"] == line["value"]
     assert line["cpu_baseline"]["kind"] == "oracle"
+
+
+@pytest.mark.parametrize("op,extra", [("insert", ["--insert-batch", "2", "--insert-tokens", "64"]),
+                                      ("absorb", ["--absorb-tokens", "2"])])
+def test_widened_rows_reference_arm(op, extra):
+    """`bench.py --op insert|absorb --impl reference`: one JSON line with the
+    contract's keys, the oracle timed on the host (no GPU needed)."""
+    cmd = [sys.executable, os.path.join(ROOT, "bench.py"), "--op", op, "--impl", "reference", "--steps", "1",
+           "--warmup", "3"] + extra
+    res = subprocess.run(cmd, cwd=ROOT, capture_output=True, text=True, timeout=600)
+    assert res.returncode == 0, res.stderr[-2000:]
+    lines = [json.loads(l) for l in res.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1, res.stdout
+    line = lines[0]
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better", "scaling",
+                "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in line, key
+    assert line["impl"] == "reference" and line["value"] > 0 and line["dtype"] == "f64"
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_insert_and_absorb_accounting():
+    """Algorithmic bytes of the widened rows, from their definitions: the
+    insert moves each token's 1152-byte row in and out plus 8 index bytes,
+    one cos/sin row per distinct position and one table entry per distinct
+    (sequence, page); the projections read each weight half once."""
+    bench = _bench()
+    sys.path.insert(0, ROOT)
+    from mla_latent_kv_26_b200.workloads import insert_inputs
+
+    d = insert_inputs(lens=[130, 70], new_tokens=[130, 6], seed=1)
+    acc = bench.insert_accounting(d)
+    pages = 3 + 1  # positions 0..129 of sequence 0 span 3 pages, 64..69 of sequence 1 one page
+    assert acc["tokens"] == 136
+    assert acc["bytes"] == 136 * (2 * 1152 + 8) + 130 * 256 + pages * 4 + 1024
+    a = bench.absorb_accounting(64, 128)
+    assert a["absorb"] == 128 * 128 * 512 * 2 + 64 * 128 * (192 + 576) * 2
+    assert a["unabsorb"] == 128 * 128 * 512 * 2 + 64 * 128 * (512 + 128) * 2
+    assert a["flops"] == 2 * 2 * 64 * 128 * 128 * 512
