@@ -28,6 +28,9 @@ Modules:
 * :mod:`oracle.cache_insert` — the step before decode: kv_norm (RMSNorm) of the
   latent, the rotary embedding of the rope key, and the write into the token's
   row of the paged cache.
+* :mod:`oracle.fp8_cache` — the fp8 (e4m3) form of the cached latent: per-token
+  scale, e4m3 rounding, and the round trip back to bf16 that an fp8-cache
+  decode sees.
 
 Pins (tests/test_oracle.py): absorption equivalence against the unabsorbed
 path, single-key exactness, probabilities summing to one, brute force with
@@ -56,3 +59,4 @@ from .decode import (  # noqa: F401
 )
 from .plan import split_plan  # noqa: F401
 from .cache_insert import rms_norm, rope_pairs, cache_insert  # noqa: F401,E402
+from .fp8_cache import e4m3_round, quantize_rows, dequantize_rows, fp8_roundtrip_cache  # noqa: F401,E402
