@@ -173,6 +173,9 @@ extern "C" MLA_API mla_status_t mla_cache_insert(const mla_insert_desc_t* desc, 
       desc->max_positions < 1 || !(desc->eps >= 0.0f) || !isfinite(desc->eps))
     return MLA_ERR_INVALID_ARG;
   if (desc->d_latent != kDLatent || desc->d_rope != kDRope || desc->page_size != kPage) return MLA_ERR_UNSUPPORTED;
+  // positions and cache rows are 32-bit in the kernel
+  if ((long long)desc->max_pages_per_seq * kPage > 0x7fffffffLL || (long long)desc->num_pages * kPage > 0x7fffffffLL)
+    return MLA_ERR_UNSUPPORTED;
   if (desc->num_tokens == 0) return MLA_OK;
   if (!kv || !weight || !cos_table || !sin_table || !seq_ids || !positions || !block_table || !kv_cache)
     return MLA_ERR_INVALID_ARG;

@@ -100,6 +100,7 @@ def _idesc(libmla, **kw):
     (dict(num_tokens=-1), 1), (dict(batch=-1), 1), (dict(max_pages_per_seq=0), 1), (dict(num_pages=0), 1),
     (dict(max_positions=0), 1), (dict(eps=-1e-6), 1), (dict(eps=float("nan")), 1), (dict(eps=float("inf")), 1),
     (dict(d_latent=256), 2), (dict(d_rope=32), 2), (dict(page_size=16), 2),
+    (dict(max_pages_per_seq=(1 << 25) + 1), 2), (dict(num_pages=(1 << 25) + 1), 2),
 ])
 def test_cache_insert_bad_descriptors_rejected(libmla, kw, status):
     d = _idesc(libmla, **kw)
