@@ -64,7 +64,9 @@ typedef struct CUstream_st* mla_stream_t;
 typedef enum {
   MLA_OK = 0,
   MLA_ERR_INVALID_ARG = 1,         /* NULL / misaligned pointer, negative size, bad flag */
-  MLA_ERR_UNSUPPORTED = 2,         /* valid but not implemented (e.g. H > 128, d_latent != 512) */
+  MLA_ERR_UNSUPPORTED = 2,         /* valid but not implemented (e.g. H > 128, d_latent != 512, or
+                                      B * Sq * max_pages_per_seq (dense) / B * Sq * ceil(topk / 64)
+                                      (sparse) pages of work at or above 2^31) */
   MLA_ERR_WORKSPACE_TOO_SMALL = 3, /* plan or workspace buffer smaller than the sizing query says */
   MLA_ERR_CUDA = 4,                /* a CUDA runtime/driver call failed */
   MLA_ERR_DEVICE_BOUNDS = 5,       /* mla_get_error: bad length, page id or index seen on device */
@@ -156,10 +158,13 @@ MLA_API mla_status_t mla_get_error(const void* plan, uint32_t* error_bits, mla_s
  *   read, so nothing has to start at zero; the array keeps the last call's
  *   contents. All calls share it: calls that overlap on the GPU (other
  *   streams, other threads) race and give wrong results. Serialise them.
- * - If the plan plus the worst-case partials (one per worker and task, at
- *   H x 2 KiB each) do not fit, fewer workers are used; if even one worker
- *   does not fit (roughly more than 120 query tokens of 128 heads per call),
- *   returns MLA_ERR_WORKSPACE_TOO_SMALL before any launch.
+ * - Limit: with T = batch * q_len query tokens, the call fits when
+ *     round_up(mla_plan_bytes(desc), 256) + (T + 1) * H * 2056 <= 32 MiB
+ *   (the plan, then one fp32 partial slot of H x 512 outputs and 2 x H LSEs
+ *   per task plus one per worker). Beyond it the call returns
+ *   MLA_ERR_WORKSPACE_TOO_SMALL before touching the device (126 query tokens
+ *   of 128 heads fit, 127 do not); within it, fewer workers are used when
+ *   the worst-case partials of all of them would not fit.
  * - Device-side errors are handled as in mla_decode (bad tokens skipped) but
  *   the error word is not reachable by the caller; use the allocating entry
  *   points to read it. */

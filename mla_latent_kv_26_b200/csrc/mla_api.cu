@@ -90,6 +90,11 @@ mla_status_t check_desc(const mla_decode_desc_t* d) {
   const long long rows = (long long)d->num_pages * kPage;
   if (tasks > (1 << 24) || rows > 0x7fffffffLL || (long long)d->max_pages_per_seq * kPage > 0x7fffffffLL)
     return MLA_ERR_UNSUPPORTED;
+  // The plan kernel lays every task's pages end to end in 32-bit prefix sums:
+  // the largest total a descriptor allows must stay below 2^31.
+  const long long pages_per_task =
+      d->topk > 0 ? ((long long)d->topk + kPage - 1) / kPage : (long long)d->max_pages_per_seq;
+  if (tasks * pages_per_task > 0x7fffffffLL) return MLA_ERR_UNSUPPORTED;
   return MLA_OK;
 }
 
@@ -311,6 +316,22 @@ bool noalloc_scratch(void** out) {
 
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
+// Scratch layout: [plan | partial outputs | partial LSEs]. The split partials
+// need one slot per (worker, task) overlap, worst case workers + tasks. The
+// call fits when the plan plus tasks + 1 slots (one worker) fit; then up to
+// *max_workers workers do. Every quantity is compared before it is
+// subtracted, so no size can wrap.
+bool noalloc_fit(const mla_decode_desc_t* desc, long long* max_workers) {
+  const size_t plan = align256(plan_bytes_for(desc));
+  const size_t per_slot = part_o_bytes(1, desc->num_heads) + part_lse_bytes(1, desc->num_heads);
+  const long long tasks = (long long)desc->batch * desc->q_len;
+  if (plan >= kNoAllocScratchBytes) return false;
+  const long long slots = (long long)((kNoAllocScratchBytes - plan) / per_slot);
+  if (slots < tasks + 1) return false;
+  *max_workers = slots - tasks;
+  return true;
+}
+
 }  // namespace
 }  // namespace mla
 
@@ -326,21 +347,18 @@ extern "C" mla_status_t mla_decode_noalloc(const mla_decode_desc_t* desc, const 
   if (!aligned16(q) || !aligned16(kv_cache) || !aligned16(out) || ((uintptr_t)lse & 3u) ||
       ((uintptr_t)block_table & 3u) || ((uintptr_t)seq_lens & 3u) || ((uintptr_t)topk_indices & 3u))
     return MLA_ERR_INVALID_ARG;  // checked here so that nothing is launched for a bad call
+  // Sizing first, on the host alone: nothing touches the device for a call
+  // whose plan and partials cannot fit.
+  long long max_workers = 0;
+  if (!noalloc_fit(desc, &max_workers)) return MLA_ERR_WORKSPACE_TOO_SMALL;
   DeviceInfo info;
   if (!device_info(&info)) return MLA_ERR_CUDA;
   void* scratch = nullptr;
   if (!noalloc_scratch(&scratch)) return MLA_ERR_CUDA;
 
-  // Scratch layout: [plan | partial outputs | partial LSEs]. The split
-  // partials need one slot per (worker, task) overlap, worst case
-  // workers + tasks; use fewer workers when that does not fit.
   const size_t plan_bytes = plan_bytes_for(desc);
-  const size_t per_slot = part_o_bytes(1, desc->num_heads) + part_lse_bytes(1, desc->num_heads);
-  const long long tasks = (long long)desc->batch * desc->q_len;
-  const long long max_slots = (long long)((kNoAllocScratchBytes - align256(plan_bytes)) / per_slot);
   long long workers = workers_for(desc, info);
-  if (workers + tasks > max_slots) workers = max_slots - tasks;
-  if (workers < 1) return MLA_ERR_WORKSPACE_TOO_SMALL;  // batch too large for the fixed scratch
+  if (workers > max_workers) workers = max_workers;
 
   mla_decode_desc_t d = *desc;
   d.num_sms = (int32_t)(2 * workers);

@@ -170,3 +170,57 @@ def test_binding_fails_loudly_without_library():
     code = "import mla_latent_kv_26_b200.binding"
     r = subprocess.run([sys.executable, "-c", code], cwd=ROOT, env=env, capture_output=True, text=True)
     assert r.returncode != 0 and "libmla.so is not built" in r.stderr
+
+
+# ---------------------------------------------------------------- limits checked on the host alone
+
+
+@pytest.mark.parametrize("kw", [
+    dict(batch=1 << 20, max_pages_per_seq=4096),                 # 2^32 pages of dense work
+    dict(batch=1 << 24, max_pages_per_seq=128),                  # 2^31
+    dict(batch=1 << 24, topk=256 * 64),                          # sparse: 2^24 tasks x 256 pages
+])
+def test_page_total_beyond_32_bits_rejected(libmla, kw):
+    """The plan kernel sums every task's pages in 32-bit prefixes: a
+    descriptor whose largest total reaches 2^31 is rejected up front."""
+    d = _desc(libmla, **kw)
+    assert libmla.mla_plan_bytes(d) == 0
+    assert libmla.mla_decode_plan(d, 16, 16, 1 << 40, None) == libmla.MLA_ERR_UNSUPPORTED
+    assert libmla.mla_decode_noalloc(d, 16, 16, 16, 16, 16, 16, 16, None) == libmla.MLA_ERR_UNSUPPORTED
+
+
+def test_page_total_just_below_32_bits_accepted(libmla):
+    d = _desc(libmla, batch=(1 << 24) - 1, max_pages_per_seq=128)   # (2^24 - 1) * 128 < 2^31
+    assert libmla.mla_plan_bytes(d) > 0
+
+
+def _noalloc_fits(T, H, plan_bytes):
+    """The documented limit: round_up(plan, 256) + (T + 1) * H * 2056 <= 32 MiB."""
+    return ((plan_bytes + 255) // 256) * 256 + (T + 1) * H * 2056 <= 32 << 20
+
+
+@pytest.mark.parametrize("batch,heads", [(1 << 22, 1), (1 << 24, 1), (127, 128), (400, 128), (16256, 1),
+                                         (2039, 8)])
+def test_noalloc_too_large_rejected_before_the_device(libmla, batch, heads):
+    """mla_decode_noalloc sizes its fixed 32 MiB scratch on the host before any
+    CUDA call: a plan that alone exceeds it (4M and 16M query tokens of one
+    head) or partials that do not fit give MLA_ERR_WORKSPACE_TOO_SMALL, with
+    dummy pointers and no GPU."""
+    d = _desc(libmla, batch=batch, num_heads=heads, max_pages_per_seq=1)
+    assert not _noalloc_fits(batch, heads, libmla.mla_plan_bytes(d))
+    assert libmla.mla_decode_noalloc(d, 16, 16, 16, 16, 16, 16, 16, None) == libmla.MLA_ERR_WORKSPACE_TOO_SMALL
+
+
+@pytest.mark.parametrize("batch,heads", [(126, 128), (16255, 1), (2038, 8)])
+def test_noalloc_largest_fitting_batch_passes_the_size_check(libmla, batch, heads):
+    d = _desc(libmla, batch=batch, num_heads=heads, max_pages_per_seq=1)
+    assert _noalloc_fits(batch, heads, libmla.mla_plan_bytes(d))
+    assert not _noalloc_fits(batch + 1, heads, libmla.mla_plan_bytes(_desc(libmla, batch=batch + 1,
+                                                                             num_heads=heads,
+                                                                             max_pages_per_seq=1)))
+    import torch
+
+    if torch.cuda.is_available():
+        pytest.skip("past the size check the call launches kernels; dummy pointers only without a GPU")
+    st = libmla.mla_decode_noalloc(d, 16, 16, 16, 16, 16, 16, 16, None)
+    assert st == libmla.MLA_ERR_CUDA        # reached the device set-up: no GPU here

@@ -3,7 +3,8 @@
 Some callers cannot call cudaMalloc while they run (a caching allocator that
 owns all device memory, or a host that forbids allocation while serving), so
 this entry point keeps its scratch in a fixed array inside the library. Here
-it is called through the C ABI twice in a row, on two different problems, and
+it is called through the C ABI three times in a row, on three different problems (the
+last one too large for all workers' partials, so it runs on fewer), and
 each result is compared with the allocating entry points (plan + decode +
 combine with caller-provided buffers) within the parity tolerances used
 elsewhere: relative L2 <= 5e-3, |a - b| <= 1e-2 + 2^-8 |b| elementwise, LSE
@@ -49,11 +50,15 @@ def test_noalloc_matches_allocating_path_twice(libmla):
 
     B = libmla
     dev = torch.device("cuda", torch.cuda.current_device())
+    lens64 = [int(x) for x in torch.randint(1, 400, (64,), generator=torch.Generator().manual_seed(73))]
     problems = [
         small(batch=4, heads=128, lens=[5000, 64, 1, 2100], seed=71, nan_tail=True),
         small(batch=3, heads=16, q_len=2, causal=True, lens=[700, 2, 4097], seed=72),
+        # 64 query tokens of 128 heads: the fixed scratch holds the partials of
+        # only 63 workers, so this call runs on fewer workers than the device has
+        small(batch=64, heads=128, lens=lens64, seed=73, nan_tail=True),
     ]
-    for d in problems:   # two calls in a row; the second reuses the scratch the first left behind
+    for d in problems:   # calls in a row; each reuses the scratch the previous one left behind
         out, lse = _noalloc(B, d, dev)
         g = _to(d, dev)
         dec = decoder_for(d, device=dev)
