@@ -38,7 +38,6 @@ UNIT = "KV-tokens/s"
 BYTES_PER_TOKEN = 576 * 2       # one cached row: c_kv[512] + k_pe[64], bf16
 FLOPS_PER_ROW_TOKEN = 2 * (576 + 512)  # QK^T over 576 + PV over 512, multiply-add = 2
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-DECODE_SRC = os.path.join(ROOT, "mla_latent_kv_26_b200", "csrc", "mla_decode.cu")
 
 
 # ---------------------------------------------------------------- accounting
@@ -72,6 +71,31 @@ def accounting(inp: dict) -> dict:
             "d2h_bytes": rows * 512 * 2 + rows * 4}
 
 
+L2_NOMINAL_BYTES = 126 * 1024 * 1024  # B200 L2, used when no device is visible (CPU reference arm)
+
+
+def l2_bytes_of(dev=None) -> int:
+    if dev is not None:
+        return int(torch.cuda.get_device_properties(dev).L2_cache_size)
+    if torch.cuda.is_available():
+        return int(torch.cuda.get_device_properties(0).L2_cache_size)
+    return L2_NOMINAL_BYTES
+
+
+def decode_config(inp: dict, acc: dict, n_gpus: int, l2_bytes: int) -> dict:
+    """The ``config`` object of the decode line; both arms print the same one."""
+    w = inp["workload"]
+    flush = acc["bytes"] < 2 * l2_bytes
+    return {"workload": f"{w.key} {w.name}", "batch": w.batch, "q_len": w.q_len, "heads": w.heads,
+            "kv_len": f"{w.len_lo}..{w.len_hi}" + (f" top{w.topk}" if w.topk else ""),
+            "kv_tokens_per_step": acc["kv_tokens"], "bytes_per_step": acc["bytes"],
+            "flops_per_step": acc["flops"], "seed": w.seed,
+            "l2": (f"{acc['bytes'] / 1e6:.0f} MB read per step, within 2x L2 ({l2_bytes / 1e6:.0f} MB): "
+                   f"L2 flushed by a {2 * l2_bytes / 1e6:.0f} MB write before every timed step")
+            if flush else f"inputs larger than 2x L2 ({acc['bytes'] / 1e6:.0f} MB read per step), no flush",
+            "parallelism": f"replicas x{n_gpus}"}
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -82,11 +106,8 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-DECODE_SOURCES = ("mla_decode.cu", "sm100.cuh", "common.cuh")
-INSERT_SOURCES = ("mla_insert.cu", "sm100.cuh", "common.cuh")
-
-
-def decode_source_sha(files=DECODE_SOURCES) -> str:
+def source_sha(files) -> str:
+    """First 16 hex digits of the sha256 of the kernel's source files, in order."""
     h = hashlib.sha256()
     for f in files:
         with open(os.path.join(ROOT, "mla_latent_kv_26_b200", "csrc", f), "rb") as fh:
@@ -94,19 +115,18 @@ def decode_source_sha(files=DECODE_SOURCES) -> str:
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(workload: str, kernel: str = "mla_decode_kernel", files=DECODE_SOURCES):
-    """DRAM bytes per launch from the committed ncu summary, if it was taken on
-    the current kernel source; else None."""
-    path = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.md")
+def profiled_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch of ``kernel`` on ``workload`` from
+    profiles/traffic.json, if that capture was taken on the current kernel
+    source; else None."""
     try:
-        text = open(path).read()
-    except OSError:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            entry = json.load(f).get(f"{kernel}/{workload}")
+    except (OSError, ValueError):
         return None
-    m_sha = re.search(r"source_sha:\s*([0-9a-f]+)", text)
-    m_b = re.search(r"dram_bytes_per_launch:\s*([0-9]+)", text)
-    if not m_sha or not m_b or m_sha.group(1) != decode_source_sha(files):
+    if not entry or entry.get("source_sha") != source_sha(entry["sources"]):
         return None
-    return int(m_b.group(1))
+    return int(entry["dram_bytes_per_launch"])
 
 
 # ---------------------------------------------------------------- clocks
@@ -219,12 +239,11 @@ def run_reference(args, inp, rank):
             secs_total += dt
             per_step.append(dt)
     value = toks_total / secs_total if secs_total > 0 else 0.0
-    w = inp["workload"]
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs_total / max(args.steps, 1),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": f"{w.key} {w.name}", "batch": w.batch, "heads": w.heads, "q_len": w.q_len},
+        "config": decode_config(inp, accounting(inp), args.gpus, l2_bytes_of()),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": torch.get_num_threads(), "kind": "oracle",
                          "sample": "float64 CPU oracle, two whole sequences of the batch per step"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -392,7 +411,7 @@ def run_insert_bench(args, world, rank, local):
                        parallelism=f"replicas x{world}"),
         "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": gbs / peaks["hbm_gbs"], "kernel": "mla_insert_kernel",
-                     "traffic": profiled_traffic(f"prefill{B}x{T}", "mla_insert_kernel", INSERT_SOURCES),
+                     "traffic": profiled_traffic("mla_insert_kernel", f"prefill{B}x{T}"),
                      "peak_source": peak_src},
         "e2e": {"value": world * acc["tokens"] / (e2e_ms / 1e3), "unit": INSERT_UNIT,
                 "h2d_bytes_per_step": acc["h2d_bytes"], "d2h_bytes_per_step": acc["d2h_bytes"], "ms_per_step": e2e_ms},
@@ -645,7 +664,7 @@ def main():
 
     # Inputs within twice the L2 size are flushed from L2 before every timed
     # step (a write of a buffer twice the L2 size, outside the step's events).
-    l2_bytes = torch.cuda.get_device_properties(dev).L2_cache_size
+    l2_bytes = l2_bytes_of(dev)
     flush_l2 = acc["bytes"] < 2 * l2_bytes
     flush_buf = torch.empty(2 * l2_bytes, dtype=torch.uint8, device=dev) if flush_l2 else None
 
@@ -663,11 +682,11 @@ def main():
     K = args.steps
     sampler = ClockSampler(local) if not args.profile else None
 
-    # K timed steps. Every eighth step also records an event between every
-    # two kernels (each such event adds a launch gap, so the other steps carry
-    # none); those steps give each kernel's own time, in the same run and
-    # thermal state as the headline.
-    SAMPLE = 8
+    # K timed steps. Every other step also records an event between every two
+    # kernels (each such event adds a launch gap, so the other steps carry
+    # none); those steps give each kernel's own time (median), in the same run
+    # and thermal state as the headline.
+    SAMPLE = 2
     sampled = [i for i in range(K) if i % SAMPLE == 0]
     kev = {i: tuple(torch.cuda.Event(enable_timing=True) for _ in range(4)) for i in sampled}
     sev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
@@ -691,11 +710,25 @@ def main():
     barrier()
     # with the L2 flush, the timed work is the sum of the steps' own intervals
     elapsed_ms = sum(a.elapsed_time(b) for a, b in sev) if flush_l2 else t_start.elapsed_time(t_end)
-    plan_ms = sum(e[0].elapsed_time(e[1]) for e in kev.values()) / len(kev)
-    decode_ms = sum(e[1].elapsed_time(e[2]) for e in kev.values()) / len(kev)
-    combine_ms = sum(e[2].elapsed_time(e[3]) for e in kev.values()) / len(kev)
+    plan_ms = statistics.median(e[0].elapsed_time(e[1]) for e in kev.values())
+    decode_ms = statistics.median(e[1].elapsed_time(e[2]) for e in kev.values())
+    combine_ms = statistics.median(e[2].elapsed_time(e[3]) for e in kev.values())
     elapsed_ms, decode_ms, plan_ms, combine_ms = max_over_ranks([elapsed_ms, decode_ms, plan_ms, combine_ms], world, dev)
     ms_per_step = elapsed_ms / K
+
+    # 100 more steps, each with an event between every two kernels, right
+    # after the timed region (not part of the headline): per-kernel medians of 100
+    K100 = 100
+    kev100 = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(4)) for _ in range(K100)]
+    barrier()
+    for i in range(K100):
+        if flush_l2:
+            flush_buf.fill_(i & 0xFF)
+        step(kev100[i])
+    torch.cuda.synchronize(dev)
+    barrier()
+    med100 = [statistics.median(e[a].elapsed_time(e[a + 1]) for e in kev100) for a in range(3)]
+    med100 = max_over_ranks(med100, world, dev)
 
     if args.profile:
         if rank == 0:
@@ -803,7 +836,7 @@ def main():
     else:
         roof = {"bound": "tensor", "achieved": achieved_tf, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                 "frac": achieved_tf / peaks["bf16_tflops"]}
-    roof["traffic"] = profiled_traffic(args.workload)
+    roof["traffic"] = profiled_traffic("mla_decode_kernel", args.workload)
     roof["peak_source"] = f"{peak_src} (MEASURED_PEAKS.json burst figures)" if peak_src == "measured" else peak_src
     roof["kernel"] = "mla_decode_kernel"
     roof["roofline_time_us"] = max(t_hbm, t_tc) * 1e6
@@ -815,19 +848,12 @@ def main():
     roof["tensor_frac"] = achieved_tf / peaks["bf16_tflops"]
 
     value = job_value(world, acc["kv_tokens"], ms_per_step)
-    w = inp["workload"]
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
         "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": f"{w.key} {w.name}", "batch": w.batch, "q_len": w.q_len, "heads": w.heads,
-                   "kv_len": f"{w.len_lo}..{w.len_hi}" + (f" top{w.topk}" if w.topk else ""),
-                   "kv_tokens_per_step": acc["kv_tokens"], "bytes_per_step": acc["bytes"],
-                   "flops_per_step": acc["flops"], "seed": w.seed, "workers": dec.num_workers,
-                   "l2": (f"{acc['bytes'] / 1e6:.0f} MB read per step, within 2x L2 ({l2_bytes / 1e6:.0f} MB): "
-                          f"L2 flushed by a {2 * l2_bytes / 1e6:.0f} MB write before every timed step")
-                   if flush_l2 else f"inputs larger than 2x L2 ({acc['bytes'] / 1e6:.0f} MB read per step), no flush",
-                   "parallelism": f"replicas x{world}"},
+        "config": decode_config(inp, acc, world, l2_bytes),
+        "launch": {"decode_workers": dec.num_workers, "ctas_per_worker": 2},
         "roofline": roof,
         "e2e": {"value": job_value(world, acc["kv_tokens"], e2e_ms), "unit": UNIT,
                 "h2d_bytes_per_step": acc["h2d_bytes"], "d2h_bytes_per_step": acc["d2h_bytes"],
@@ -836,7 +862,9 @@ def main():
                         "back every step; consecutive steps alternate between two decoders on two streams"},
         "gpu_launches": 3 * K,
         "kernels_us": {"plan": plan_ms * 1e3, "decode": decode_ms * 1e3, "combine": combine_ms * 1e3,
-                       "sampled_steps": len(kev)},
+                       "sampled_steps": len(kev), "statistic": "median of the sampled timed steps",
+                       "median_of_100_after": {"plan": med100[0] * 1e3, "decode": med100[1] * 1e3,
+                                               "combine": med100[2] * 1e3}},
         "graph_ms_per_step": graph_ms,
         "clocks": sampler.summary() if sampler else None,
     }

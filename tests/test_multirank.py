@@ -85,6 +85,15 @@ def test_reference_arm_under_torchrun_two_ranks():
     assert line["impl"] == "reference" and line["n_gpus"] == 2
     assert line["value"] > 0 and line["e2e"]["value"] == line["value"]
     assert line["cpu_baseline"]["kind"] == "oracle"
+    # the same config object the GPU arm prints for this workload (so the two
+    # lines compare as one configuration)
+    bench = _bench()
+    sys.path.insert(0, ROOT)
+    from mla_latent_kv_26_b200.workloads import make_inputs
+
+    inp = make_inputs("C1")
+    assert line["config"] == bench.decode_config(inp, bench.accounting(inp), 2, bench.l2_bytes_of())
+    assert "l2" in line["config"] and line["config"]["parallelism"] == "replicas x2"
 
 
 @pytest.mark.parametrize("op,extra", [("insert", ["--insert-batch", "2", "--insert-tokens", "64"]),

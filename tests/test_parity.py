@@ -269,18 +269,32 @@ def test_bad_sparse_index_is_skipped_and_flagged(dev):
 
 
 @pytest.mark.parametrize("key", ["C1", "C2", "C3", "C4", "C5"])
-def test_full_size_workload_sampled(dev, key):
+def test_full_size_workload(dev, key):
     """The benchmark workloads at full size in the benchmark's launch
-    configuration (all SMs); the oracle checks a sample of sequences (the
-    shortest, the longest and one more), the rest must be finite."""
+    configuration (all SMs): every sequence of the batch against the oracle,
+    element by element, with the relative L2 error taken over the whole
+    output tensor."""
     from mla_latent_kv_26_b200.workloads import make_inputs
 
     d = make_inputs(key)
     out, lse, st, bits, dec = run_gpu(d, dev, 0)
     assert st == 0 and bits == 0
     assert torch.isfinite(out).all() and torch.isfinite(lse).all()
-    lens = d["seq_lens"].tolist()
-    pick = sorted({lens.index(min(lens)), lens.index(max(lens)), len(lens) // 2})
     o_ref, l_ref = oracle.mla_decode(d["q"], d["cache"], d["block_table"], d["seq_lens"], causal=d["causal"],
-                                     indices=d["indices"], batches=pick)
-    assert_parity(out[pick], lse[pick], o_ref[pick], l_ref[pick], key)
+                                     indices=d["indices"])
+    assert_parity(out, lse, o_ref, l_ref, key)
+
+
+@pytest.mark.parametrize("q_std", [10.0, 20.0])
+@pytest.mark.parametrize("heads", [128, 16])
+def test_large_magnitude_queries(dev, q_std, heads):
+    """Queries 10x and 20x the usual scale against an N(0, 1) cache: partial
+    scores of each CTA half reach the hundreds, where the 16-bit block
+    fixed-point exchange of partial scores is coarsest (its error per score is
+    at most 2^-15 of the largest partial score of the row in the tile). Both
+    the output and the LSE must stay within the usual tolerances."""
+    from mla_latent_kv_26_b200.workloads import small
+
+    d = small(batch=4, heads=heads, lens=[3000, 700, 64, 1], seed=int(q_std) + heads, q_std=q_std)
+    check_case(d, dev, 0, f"q std {q_std} H{heads}")
+    check_case(d, dev, 2, f"q std {q_std} H{heads} one worker")
