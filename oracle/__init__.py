@@ -31,6 +31,9 @@ Modules:
 * :mod:`oracle.fp8_cache` — the fp8 (e4m3) form of the cached latent: per-token
   scale, e4m3 rounding, and the round trip back to bf16 that an fp8-cache
   decode sees.
+* :mod:`oracle.indexer` — the sparse-attention indexer ("DeepSeek-V3.2-Exp
+  unboxing", the Indexer section): fp8 index scores per (query, key) and the
+  top-k positions that the sparse decode attends to.
 
 Pins (tests/test_oracle.py): absorption equivalence against the unabsorbed
 path, single-key exactness, probabilities summing to one, brute force with
@@ -60,3 +63,4 @@ from .decode import (  # noqa: F401
 from .plan import split_plan  # noqa: F401
 from .cache_insert import rms_norm, rope_pairs, cache_insert  # noqa: F401,E402
 from .fp8_cache import e4m3_round, quantize_rows, dequantize_rows, fp8_roundtrip_cache  # noqa: F401,E402
+from .indexer import index_scores, topk_positions  # noqa: F401,E402
