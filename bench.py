@@ -590,6 +590,167 @@ def run_absorb_bench(args, world, rank, local):
         dist.destroy_process_group()
 
 
+# ---------------------------------------------------------------- indexer + top-k (--op indexer)
+
+INDEXER_METRIC = ("sparse-attention indexer keys/s (fp8 index scores + exact top-k) and achieved GB/s vs HBM "
+                  "roofline")
+INDEXER_UNIT = "keys/s"
+
+
+def indexer_accounting(b: int, m: int, h: int, n: int, k: int) -> dict:
+    """Algorithmic bytes: the scores kernel reads q, q_s, k and k_s once and
+    writes the scores; the top-k reads the scores and writes the positions."""
+    scores = b * m * h * 128 + 4 * b * m * h + b * n * 128 + 4 * b * n + 4 * b * m * n
+    topk = 4 * b * m * n + 4 * b * m * k
+    flops = 2 * b * m * h * n * 128
+    return {"scores": scores, "topk": topk, "bytes": scores + topk, "flops": flops, "keys": b * m * n,
+            "h2d_bytes": b * m * h * (128 + 4), "d2h_bytes": 4 * b * m * k}
+
+
+def indexer_oracle_sample(d: dict, k: int, budget_s: float):
+    """The oracle's scores and top-k for whole query rows until the budget is
+    used; returns (keys scored, seconds)."""
+    import oracle
+
+    t0, done, r = time.perf_counter(), 0, 0
+    while time.perf_counter() - t0 < budget_s:
+        b = r % d["batch"]
+        sc = oracle.index_scores(d["q"][b:b + 1], d["q_s"][b:b + 1], d["k"][b:b + 1], d["k_s"][b:b + 1])
+        oracle.topk_positions(sc.view(-1, d["num_keys"]), k)
+        done += d["q_len"] * d["num_keys"]
+        r += 1
+    return done, time.perf_counter() - t0
+
+
+def run_indexer_bench(args, world, rank, local):
+    from mla_latent_kv_26_b200.workloads import indexer_inputs
+
+    b, m, h, n, K = 16, 1, 64, 131072, 2048
+    d = indexer_inputs(batch=b, q_len=m, heads=h, num_keys=n, seed=8)
+    acc = indexer_accounting(b, m, h, n, K)
+    cfg = {"workload": f"indexer-b{b}-m{m}-h{h}-n{n}-top{K}: fp8 index scores of {n} keys for {b} sequences, "
+                       f"{h} index heads of 128, then the top {K} positions per query",
+           "keys_per_step": acc["keys"], "bytes_per_step": acc["bytes"], "flops_per_step": acc["flops"],
+           "l2": f"inputs larger than 2x L2 ({acc['bytes'] / 1e6:.0f} MB moved per step), no flush",
+           "parallelism": f"replicas x{args.gpus if args.impl == 'reference' else world}"}
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        torch.set_num_threads(os.cpu_count() or 1)
+        keys, secs = 0, 0.0
+        for s in range(args.warmup + args.steps):
+            kk, dt = indexer_oracle_sample(d, K, 0.3)
+            if s >= args.warmup:
+                keys, secs = keys + kk, secs + dt
+        v = keys / secs
+        print(json.dumps({
+            "impl": "reference", "metric": INDEXER_METRIC, "value": v, "unit": INDEXER_UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": cfg,
+            "cpu_baseline": {"value": v, "unit": INDEXER_UNIT, "cores": torch.get_num_threads(), "kind": "oracle",
+                             "sample": "float64 oracle scores + top-k of whole query rows, about 0.3 s per step"},
+            "e2e": {"value": v, "unit": INDEXER_UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}),
+              flush=True)
+        return
+
+    import torch.distributed as dist
+
+    from mla_latent_kv_26_b200 import binding as Bd
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+    g = {key: (v.to(dev) if isinstance(v, torch.Tensor) else v) for key, v in d.items()}
+    scores = torch.empty(b, m, n, dtype=torch.float32, device=dev)
+    idx = torch.empty(b * m, K, dtype=torch.int32, device=dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    lens = torch.full((b * m,), n, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    sdesc = Bd.make_index_desc(batch=b, q_len=m, num_heads=h, num_keys=n)
+    tdesc = Bd.make_topk_desc(rows=b * m, num_keys=n, k=K)
+
+    def step(q, q_s, ev=None, st=stream):
+        if ev is not None:
+            ev[0].record(st)
+        Bd.check(Bd.mla_index_scores(sdesc, q, q_s, g["k"], g["k_s"], scores, err, st), "mla_index_scores")
+        if ev is not None:
+            ev[1].record(st)
+        Bd.check(Bd.mla_topk(tdesc, scores, lens, idx, st), "mla_topk")
+        if ev is not None:
+            ev[2].record(st)
+
+    for _ in range(args.warmup):
+        step(g["q"], g["q_s"])
+    torch.cuda.synchronize(dev)
+    K_steps = args.steps
+    ev = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(3)) for _ in range(K_steps)]
+    sampler = ClockSampler(local, interval_s=0.002)
+    if world > 1:
+        dist.barrier(device_ids=[local])
+    torch.cuda.synchronize(dev)
+    with sampler:
+        for i in range(K_steps):
+            step(g["q"], g["q_s"], ev[i])
+        torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier(device_ids=[local])
+    s_ms = statistics.median(e[0].elapsed_time(e[1]) for e in ev)
+    t_ms = statistics.median(e[1].elapsed_time(e[2]) for e in ev)
+    ms = sum(e[0].elapsed_time(e[2]) for e in ev) / K_steps
+    ms, s_ms, t_ms = max_over_ranks([ms, s_ms, t_ms], world, dev)
+    if int(err.item()) != 0:
+        raise RuntimeError(f"device error word {int(err.item()):#x}")
+
+    # end to end: the step's queries and weights in from pinned host memory,
+    # the chosen positions back, every step (the key cache stays resident)
+    hq, hqs = d["q"].pin_memory(), d["q_s"].pin_memory()
+    hidx = torch.empty(b * m, K, dtype=torch.int32).pin_memory()
+    dq, dqs = torch.empty_like(g["q"]), torch.empty_like(g["q_s"])
+    K2 = max(3, min(K_steps, 50))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    for _ in range(K2):
+        dq.copy_(hq, non_blocking=True)
+        dqs.copy_(hqs, non_blocking=True)
+        step(dq, dqs)
+        hidx.copy_(idx, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    (e2e_ms,) = max_over_ranks([e0.elapsed_time(e1) / K2], world, dev)
+
+    peaks, peak_src = load_peaks()
+    s_gbs = acc["scores"] / (s_ms / 1e3) / 1e9
+    t_gbs = acc["topk"] / (t_ms / 1e3) / 1e9
+    line = {
+        "metric": INDEXER_METRIC, "value": world * acc["keys"] / (ms / 1e3), "unit": INDEXER_UNIT, "n_gpus": world,
+        "steps": K_steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "e4m3 in, f32 accumulate", "data": "synthetic", "config": cfg,
+        "roofline": {"bound": "hbm", "achieved": s_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": s_gbs / peaks["hbm_gbs"], "kernel": "mla_index_kernel",
+                     "traffic": profiled_traffic("mla_index_kernel", f"b{b}n{n}"), "peak_source": peak_src,
+                     "scores_us": s_ms * 1e3, "topk_us": t_ms * 1e3, "topk_gbs": t_gbs,
+                     "tflop_per_s": acc["flops"] / (s_ms / 1e3) / 1e12},
+        "e2e": {"value": world * acc["keys"] / (e2e_ms / 1e3), "unit": INDEXER_UNIT,
+                "h2d_bytes_per_step": acc["h2d_bytes"], "d2h_bytes_per_step": acc["d2h_bytes"], "ms_per_step": e2e_ms},
+        "gpu_launches": 2 * K_steps,
+        "clocks": sampler.summary(),
+    }
+    if rank == 0 and world == 1:
+        torch.set_num_threads(os.cpu_count() or 1)
+        kk, secs = indexer_oracle_sample(d, K, args.cpu_budget)
+        line["cpu_baseline"] = {"value": kk / secs, "unit": INDEXER_UNIT, "cores": torch.get_num_threads(),
+                                "kind": "oracle", "sample": f"{kk} keys (whole query rows), float64, {secs:.1f} s"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
 # ---------------------------------------------------------------- GPU arm
 
 
@@ -603,9 +764,9 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle time for cpu_baseline")
     ap.add_argument("--profile", action="store_true", help="kernel launches only (for ncu): no e2e/oracle/clocks")
     ap.add_argument("--num-sms", type=int, default=0)
-    ap.add_argument("--op", default="decode", choices=["decode", "insert", "absorb"],
+    ap.add_argument("--op", default="decode", choices=["decode", "insert", "absorb", "indexer"],
                     help="decode: the decode step (default); insert: the latent-cache insert alone; "
-                         "absorb: the absorb + un-absorb projections")
+                         "absorb: the absorb + un-absorb projections; indexer: fp8 index scores + top-k")
     ap.add_argument("--absorb-tokens", type=int, default=64, help="query tokens for --op absorb")
     ap.add_argument("--insert-batch", type=int, default=64)
     ap.add_argument("--insert-tokens", type=int, default=1024, help="new tokens per sequence for --op insert")
@@ -623,6 +784,9 @@ def main():
         return
     if args.op == "absorb":
         run_absorb_bench(args, world, rank, local)
+        return
+    if args.op == "indexer":
+        run_indexer_bench(args, world, rank, local)
         return
 
     inp = make_inputs(args.workload)

@@ -142,6 +142,31 @@ MLA_API mla_status_t mla_combine(const mla_decode_desc_t* desc, void* plan, cons
  * (timeout bit set) or MLA_ERR_DEVICE_BOUNDS (any other bit). */
 MLA_API mla_status_t mla_get_error(const void* plan, uint32_t* error_bits, mla_stream_t stream);
 
+/* Merge of decode results computed over disjoint token sets of the same
+ * rows: the combine step of decode context parallelism, where each of N
+ * ranks holds a shard of every sequence's cache, decodes over it, and the
+ * ranks' (out, lse) are gathered (the beaiera.top DeepSeek tag page, the
+ * abstract on DCP: the KV cache sharded along the sequence across ranks).
+ * The same LSE merge as mla_combine, over whole shard results:
+ *
+ *   lse = ln sum_i exp(lse_i),   out = sum_i exp(lse_i - lse) * out_i
+ *
+ * parts with lse_i = -inf (no visible token in that shard) weigh nothing;
+ * a row empty in every part gets out = 0, lse = -inf.
+ *   part_out  bf16 [parts, rows, 512] (each part's mla_decode output, rows = B * Sq * H)
+ *   part_lse  fp32 [parts, rows]
+ *   out       bf16 [rows, 512]     lse  fp32 [rows]
+ * part_out and out 16-byte aligned. One kernel, asynchronous on `stream`,
+ * no allocation. */
+typedef struct {
+  int32_t parts;    /* N >= 1 */
+  int32_t d_latent; /* must be 512 */
+  int64_t rows;     /* rows per part, >= 0 */
+} mla_merge_desc_t;
+
+MLA_API mla_status_t mla_merge(const mla_merge_desc_t* desc, const void* part_out, const float* part_lse, void* out,
+                               float* lse, mla_stream_t stream);
+
 /* Decode step with no device allocation by anyone: plan + decode + combine as
  * above, with the plan and the split partials kept in a fixed 32 MiB array of
  * device memory that the library itself defines (every device that loads
@@ -257,6 +282,67 @@ MLA_API mla_status_t mla_absorb_query(const mla_absorb_desc_t* desc, const void*
                                       uint32_t* error_word, mla_stream_t stream);
 MLA_API mla_status_t mla_unabsorb_output(const mla_absorb_desc_t* desc, const void* o_lat, const void* wkv_b,
                                          void* out, uint32_t* error_word, mla_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * Sparse-attention indexer: index scores and their top-k positions, the step
+ * that picks the tokens a sparse decode (desc->topk > 0) attends to.
+ *
+ * "DeepSeek-V3.2-Exp unboxing", the Indexer section: the indexer scores the
+ * cached keys of each sequence for each query token and keeps the
+ * highest-scoring positions. Its scoring kernel takes fp8_index(q [b, m, h, d]
+ * fp8, q_s [b, m, h] fp32, k [b, n, d] fp8, k_s [b, n] fp32) -> o [b, m, n]
+ * fp32, with the model's per-head weights passed as q_s and the fp8 key
+ * cache's per-token scales as k_s (shapes seen there: q [2, 128, 64, 128],
+ * k [2, 128, 128]). The page does not print the kernel body; the score here
+ * is the plain reading, a ReLU of each head's dot product weighted by q_s and
+ * summed over heads, times the key's scale:
+ *
+ *   scores[b, i, t] = k_s[b, t] * sum_h q_s[b, i, h] * max(0, sum_d q[b, i, h, d] * k[b, t, d])
+ *
+ *   q       e4m3 (1 byte: sign, 4 exponent bits with bias 7, 3 mantissa bits;
+ *           no infinities) [b, m, h, 128], 16-byte aligned
+ *   q_s     fp32 [b, m, h], 16-byte aligned
+ *   k       e4m3 [b, n, 128] (each sequence's keys contiguous), 16-byte aligned
+ *   k_s     fp32 [b, n]
+ *   scores  fp32 [b, m, n] (written for every t < n; no masking: the top-k
+ *           call below takes each row's valid length)
+ *   error_word  device uint32 or NULL: MLA_DEVERR_TIMEOUT is OR-ed in if a
+ *           bounded device wait ran out (scores then invalid)
+ * Products of two e4m3 values are exact in fp32; the sums over d (tensor
+ * cores) and over h are fp32. h must be a multiple of 16, at most 256; d must
+ * be 128. One kernel, asynchronous on `stream`, no allocation. */
+typedef struct {
+  int32_t batch;     /* b >= 0 */
+  int32_t q_len;     /* m >= 1: query tokens per sequence */
+  int32_t num_heads; /* h: index heads, a multiple of 16 in [16, 256] */
+  int32_t head_dim;  /* d: must be 128 */
+  int32_t num_keys;  /* n >= 0: keys per sequence */
+} mla_index_desc_t;
+
+MLA_API mla_status_t mla_index_scores(const mla_index_desc_t* desc, const void* q, const float* q_s, const void* k,
+                                      const float* k_s, float* scores, uint32_t* error_word, mla_stream_t stream);
+
+/* Top-k positions of each row of a score matrix, exactly (no approximation).
+ *   scores      fp32 [rows, n] (for the indexer: rows = b * m)
+ *   valid_lens  int32 [rows] or NULL: row r considers positions t < valid_lens[r]
+ *               (clamped to [0, n]); NULL = all n. For a decode step this is
+ *               seq_lens[b], or seq_lens[b] - Sq + i + 1 for causal query i.
+ *   indices     int32 [rows, k]: the k positions with the largest scores in
+ *               increasing order, equal scores at the cut going to the
+ *               smaller positions (-0.0 and +0.0 are equal); when fewer than
+ *               k positions are eligible, all of them and then -1. This is
+ *               mla_decode's topk_indices layout (-1 = skip).
+ * Scores must not be NaN (a NaN ranks above every number). Rows are
+ * independent; one kernel (a cluster of up to 8 CTAs per row), asynchronous
+ * on `stream`, no allocation. */
+typedef struct {
+  int32_t rows;     /* >= 0 */
+  int32_t num_keys; /* n >= 0: scores per row (the row stride) */
+  int32_t k;        /* >= 1: positions kept per row */
+} mla_topk_desc_t;
+
+MLA_API mla_status_t mla_topk(const mla_topk_desc_t* desc, const float* scores, const int32_t* valid_lens,
+                              int32_t* indices, mla_stream_t stream);
 
 /* Static string for a status code. */
 MLA_API const char* mla_status_string(mla_status_t status);

@@ -31,7 +31,7 @@ MLA_DEVERR_POSITION = 0x10
 EXPORTED = (
     "mla_plan_bytes", "mla_workspace_bytes", "mla_num_workers", "mla_decode_plan", "mla_decode",
     "mla_combine", "mla_get_error", "mla_status_string", "mla_decode_noalloc", "mla_cache_insert",
-    "mla_absorb_query", "mla_unabsorb_output",
+    "mla_absorb_query", "mla_unabsorb_output", "mla_index_scores", "mla_topk", "mla_merge",
 )
 
 DEFAULT_SOFTMAX_SCALE = 1.0 / math.sqrt(192.0)
@@ -98,6 +98,44 @@ def make_absorb_desc(*, num_tokens: int, num_heads: int, d_nope: int = 128, d_ro
     return mla_absorb_desc_t(num_tokens, num_heads, d_nope, d_rope, d_latent, d_v)
 
 
+class mla_index_desc_t(ctypes.Structure):
+    _fields_ = [
+        ("batch", ctypes.c_int32),
+        ("q_len", ctypes.c_int32),
+        ("num_heads", ctypes.c_int32),
+        ("head_dim", ctypes.c_int32),
+        ("num_keys", ctypes.c_int32),
+    ]
+
+
+def make_index_desc(*, batch: int, q_len: int, num_heads: int, num_keys: int, head_dim: int = 128) -> mla_index_desc_t:
+    return mla_index_desc_t(batch, q_len, num_heads, head_dim, num_keys)
+
+
+class mla_topk_desc_t(ctypes.Structure):
+    _fields_ = [
+        ("rows", ctypes.c_int32),
+        ("num_keys", ctypes.c_int32),
+        ("k", ctypes.c_int32),
+    ]
+
+
+def make_topk_desc(*, rows: int, num_keys: int, k: int) -> mla_topk_desc_t:
+    return mla_topk_desc_t(rows, num_keys, k)
+
+
+class mla_merge_desc_t(ctypes.Structure):
+    _fields_ = [
+        ("parts", ctypes.c_int32),
+        ("d_latent", ctypes.c_int32),
+        ("rows", ctypes.c_int64),
+    ]
+
+
+def make_merge_desc(*, parts: int, rows: int, d_latent: int = 512) -> mla_merge_desc_t:
+    return mla_merge_desc_t(parts, d_latent, rows)
+
+
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
         raise RuntimeError(
@@ -119,6 +157,9 @@ def _load() -> ctypes.CDLL:
         "mla_cache_insert": (ctypes.c_int, [ctypes.POINTER(mla_insert_desc_t), P, P, P, P, P, P, P, P, P, P]),
         "mla_absorb_query": (ctypes.c_int, [ctypes.POINTER(mla_absorb_desc_t), P, P, P, P, P]),
         "mla_unabsorb_output": (ctypes.c_int, [ctypes.POINTER(mla_absorb_desc_t), P, P, P, P, P]),
+        "mla_index_scores": (ctypes.c_int, [ctypes.POINTER(mla_index_desc_t), P, P, P, P, P, P, P]),
+        "mla_topk": (ctypes.c_int, [ctypes.POINTER(mla_topk_desc_t), P, P, P, P]),
+        "mla_merge": (ctypes.c_int, [ctypes.POINTER(mla_merge_desc_t), P, P, P, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -209,6 +250,23 @@ def mla_unabsorb_output(desc, o_lat, wkv_b, out, error_word=None, stream=None) -
     """o_lat [T,H,512] -> out [T,H,128] = W_UV o_lat."""
     return int(_lib.mla_unabsorb_output(ctypes.byref(desc), _ptr(o_lat), _ptr(wkv_b), _ptr(out), _ptr(error_word),
                                         _stream(stream)))
+
+
+def mla_index_scores(desc, q, q_s, k, k_s, scores, error_word=None, stream=None) -> int:
+    """fp8 index scores [b, m, n] of every key for every query token."""
+    return int(_lib.mla_index_scores(ctypes.byref(desc), _ptr(q), _ptr(q_s), _ptr(k), _ptr(k_s), _ptr(scores),
+                                     _ptr(error_word), _stream(stream)))
+
+
+def mla_topk(desc, scores, valid_lens, indices, stream=None) -> int:
+    """Top-k positions of each score row, increasing, -1 padded."""
+    return int(_lib.mla_topk(ctypes.byref(desc), _ptr(scores), _ptr(valid_lens), _ptr(indices), _stream(stream)))
+
+
+def mla_merge(desc, part_out, part_lse, out, lse, stream=None) -> int:
+    """LSE merge of per-shard decode results [parts, rows, 512] / [parts, rows]."""
+    return int(_lib.mla_merge(ctypes.byref(desc), _ptr(part_out), _ptr(part_lse), _ptr(out), _ptr(lse),
+                              _stream(stream)))
 
 
 def mla_get_error(plan, stream=None):

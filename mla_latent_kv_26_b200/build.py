@@ -17,7 +17,8 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libmla.so")
-SOURCES = ["mla_api.cu", "mla_decode.cu", "mla_plan_combine.cu", "mla_insert.cu", "mla_absorb.cu"]
+SOURCES = ["mla_api.cu", "mla_decode.cu", "mla_plan_combine.cu", "mla_insert.cu", "mla_absorb.cu",
+           "mla_indexer.cu"]
 HEADERS = ["common.cuh", "sm100.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

@@ -206,3 +206,31 @@ def absorb_inputs(*, tokens: int, heads: int, seed: int = 0, w_std: float = 0.05
     wkv_b = (torch.randn(heads, 256, 512, generator=g) * w_std).to(torch.bfloat16)
     o_lat = (torch.randn(tokens, heads, 512, generator=g) * o_std).to(torch.bfloat16)
     return {"q": q, "wkv_b": wkv_b, "o_lat": o_lat, "tokens": tokens, "heads": heads}
+
+
+def indexer_inputs(*, batch: int, q_len: int, heads: int, num_keys: int, seed: int = 0, code_std: float = 16.0,
+                   chunk: int = 1 << 22) -> dict:
+    """Inputs of the sparse-attention indexer ("DeepSeek-V3.2-Exp unboxing",
+    the Indexer section: fp8 q [b, m, h, 128] with per-head weights q_s
+    [b, m, h], fp8 keys k [b, n, 128] with per-key scales k_s [b, n]).
+
+    Draw order, from one generator: q codes -> q_s -> k codes -> k_s. Codes
+    are N(0, code_std^2) clipped to the e4m3 range and cast to e4m3 by the
+    library; q_s ~ N(0, 1/h) (weights of either sign); k_s ~ U[0.5, 1.5) /
+    code_std (positive scales)."""
+    g = torch.Generator().manual_seed(seed)
+    D = 128
+
+    def codes(n_rows):
+        out = torch.empty(n_rows, D, dtype=torch.float8_e4m3fn)
+        for r0 in range(0, n_rows, max(1, chunk // D)):
+            r1 = min(n_rows, r0 + max(1, chunk // D))
+            out[r0:r1] = (torch.randn(r1 - r0, D, generator=g) * code_std).clamp(-448, 448).to(torch.float8_e4m3fn)
+        return out
+
+    q = codes(batch * q_len * heads).view(batch, q_len, heads, D)
+    q_s = torch.randn(batch, q_len, heads, generator=g) / math.sqrt(heads)
+    k = codes(batch * num_keys).view(batch, num_keys, D)
+    k_s = (0.5 + torch.rand(batch, num_keys, generator=g)) / code_std
+    return {"q": q, "q_s": q_s, "k": k, "k_s": k_s, "batch": batch, "q_len": q_len, "heads": heads,
+            "num_keys": num_keys}

@@ -25,8 +25,8 @@ def _declared():
 def test_header_declares_the_boundary():
     assert _declared() == sorted([
         "mla_absorb_query", "mla_cache_insert", "mla_combine", "mla_decode", "mla_decode_noalloc", "mla_decode_plan",
-        "mla_get_error", "mla_num_workers", "mla_plan_bytes", "mla_status_string", "mla_unabsorb_output",
-        "mla_workspace_bytes"])
+        "mla_get_error", "mla_index_scores", "mla_merge", "mla_num_workers", "mla_plan_bytes", "mla_status_string",
+        "mla_topk", "mla_unabsorb_output", "mla_workspace_bytes"])
 
 
 def test_library_exports_every_declared_symbol(libmla):
@@ -224,3 +224,67 @@ def test_noalloc_largest_fitting_batch_passes_the_size_check(libmla, batch, head
         pytest.skip("past the size check the call launches kernels; dummy pointers only without a GPU")
     st = libmla.mla_decode_noalloc(d, 16, 16, 16, 16, 16, 16, 16, None)
     assert st == libmla.MLA_ERR_CUDA        # reached the device set-up: no GPU here
+
+
+# ---------------------------------------------------------------- indexer and top-k
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(batch=-1), 1), (dict(q_len=0), 1), (dict(num_heads=0), 1), (dict(num_keys=-1), 1),
+    (dict(head_dim=64), 2), (dict(num_heads=24), 2), (dict(num_heads=272), 2),
+    (dict(batch=1 << 16, num_keys=1 << 16), 2), (dict(batch=1 << 12, q_len=1 << 12, num_heads=256), 2),
+])
+def test_index_bad_descriptors_rejected(libmla, kw, status):
+    base = dict(batch=2, q_len=1, num_heads=64, num_keys=300)
+    base.update(kw)
+    d = libmla.make_index_desc(**base)
+    assert libmla.mla_index_scores(d, 16, 16, 16, 16, 16, None, None) == status
+
+
+def test_index_null_misaligned_and_empty(libmla):
+    d = libmla.make_index_desc(batch=2, q_len=1, num_heads=64, num_keys=300)
+    good = [16, 16, 16, 16, 16]
+    for i in range(5):
+        a = list(good)
+        a[i] = None
+        assert libmla.mla_index_scores(d, *a, None, None) == libmla.MLA_ERR_INVALID_ARG, i
+    for i, off in ((0, 8), (1, 4), (2, 8), (3, 2), (4, 2)):
+        a = list(good)
+        a[i] += off
+        assert libmla.mla_index_scores(d, *a, None, None) == libmla.MLA_ERR_INVALID_ARG, i
+    assert libmla.mla_index_scores(d, *good, 18, None) == libmla.MLA_ERR_INVALID_ARG
+    for empty in (dict(batch=0), dict(num_keys=0)):
+        e = libmla.make_index_desc(**dict(dict(batch=2, q_len=1, num_heads=64, num_keys=300), **empty))
+        assert libmla.mla_index_scores(e, None, None, None, None, None, None, None) == libmla.MLA_OK
+
+
+def test_topk_bad_arguments_rejected(libmla):
+    INV = libmla.MLA_ERR_INVALID_ARG
+    mk = libmla.make_topk_desc
+    assert libmla.mla_topk(mk(rows=-1, num_keys=8, k=2), 16, None, 16, None) == INV
+    assert libmla.mla_topk(mk(rows=2, num_keys=-1, k=2), 16, None, 16, None) == INV
+    assert libmla.mla_topk(mk(rows=2, num_keys=8, k=0), 16, None, 16, None) == INV
+    assert libmla.mla_topk(mk(rows=2, num_keys=8, k=2), None, None, 16, None) == INV
+    assert libmla.mla_topk(mk(rows=2, num_keys=8, k=2), 16, None, None, None) == INV
+    assert libmla.mla_topk(mk(rows=2, num_keys=8, k=2), 18, None, 16, None) == INV
+    assert libmla.mla_topk(mk(rows=2, num_keys=8, k=2), 16, 18, 16, None) == INV
+    assert libmla.mla_topk(mk(rows=2, num_keys=8, k=2), 16, None, 18, None) == INV
+    assert libmla.mla_topk(mk(rows=1 << 29, num_keys=8, k=2), 16, None, 16, None) == libmla.MLA_ERR_UNSUPPORTED
+    assert libmla.mla_topk(mk(rows=0, num_keys=8, k=2), None, None, None, None) == libmla.MLA_OK
+
+
+def test_merge_bad_arguments_rejected(libmla):
+    INV = libmla.MLA_ERR_INVALID_ARG
+    mk = libmla.make_merge_desc
+    assert libmla.mla_merge(mk(parts=0, rows=4), 16, 16, 16, 16, None) == INV
+    assert libmla.mla_merge(mk(parts=2, rows=-1), 16, 16, 16, 16, None) == INV
+    assert libmla.mla_merge(mk(parts=2, rows=4, d_latent=256), 16, 16, 16, 16, None) == libmla.MLA_ERR_UNSUPPORTED
+    for i in range(4):
+        a = [16, 16, 16, 16]
+        a[i] = None
+        assert libmla.mla_merge(mk(parts=2, rows=4), *a, None) == INV, i
+    for i, off in ((0, 8), (1, 2), (2, 8), (3, 2)):
+        a = [16, 16, 16, 16]
+        a[i] += off
+        assert libmla.mla_merge(mk(parts=2, rows=4), *a, None) == INV, i
+    assert libmla.mla_merge(mk(parts=2, rows=0), None, None, None, None, None) == libmla.MLA_OK
