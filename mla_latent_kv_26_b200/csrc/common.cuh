@@ -68,6 +68,15 @@ struct CombineArgs {
   int q_len, heads;
 };
 
+struct MergeArgs {
+  const __nv_bfloat16* part_out;  // [parts, rows, 512]
+  const float* part_lse;          // [parts, rows]
+  __nv_bfloat16* out;             // [rows, 512]
+  float* lse;                     // [rows]
+  int parts;
+  long long rows;
+};
+
 // Workspace layout: part_o then part_lse.
 __host__ __device__ inline size_t part_o_bytes(int slots, int heads) {
   return (size_t)slots * heads * kDLatent * sizeof(float);

@@ -13,6 +13,7 @@ namespace mla {
 
 cudaError_t launch_plan(const PlanArgs& args, cudaStream_t stream);
 cudaError_t launch_combine(const CombineArgs& args, int tasks, cudaStream_t stream);
+cudaError_t launch_merge(const MergeArgs& args, cudaStream_t stream);
 const void* decode_kernel_ptr();
 int decode_smem_bytes();
 int decode_threads();
@@ -264,6 +265,26 @@ mla_status_t mla_get_error(const void* plan, uint32_t* error_bits, mla_stream_t 
   if (bits & kErrTimeout) return MLA_ERR_DEVICE_TIMEOUT;
   if (bits) return MLA_ERR_DEVICE_BOUNDS;
   return MLA_OK;
+}
+
+mla_status_t mla_merge(const mla_merge_desc_t* desc, const void* part_out, const float* part_lse, void* out, float* lse,
+                       mla_stream_t stream) {
+  if (!desc) return MLA_ERR_INVALID_ARG;
+  if (desc->parts < 1 || desc->rows < 0) return MLA_ERR_INVALID_ARG;
+  if (desc->d_latent != kDLatent) return MLA_ERR_UNSUPPORTED;
+  if (desc->rows == 0) return MLA_OK;
+  if ((desc->rows + 7) / 8 > 0x7fffffffLL || desc->rows * desc->parts > (1LL << 40)) return MLA_ERR_UNSUPPORTED;
+  if (!part_out || !part_lse || !out || !lse) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(part_out) || !aligned16(out) || ((uintptr_t)part_lse & 3u) || ((uintptr_t)lse & 3u))
+    return MLA_ERR_INVALID_ARG;
+  MergeArgs a;
+  a.part_out = reinterpret_cast<const __nv_bfloat16*>(part_out);
+  a.part_lse = part_lse;
+  a.out = reinterpret_cast<__nv_bfloat16*>(out);
+  a.lse = lse;
+  a.parts = desc->parts;
+  a.rows = desc->rows;
+  return launch_merge(a, (cudaStream_t)stream) == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
 const char* mla_status_string(mla_status_t s) {

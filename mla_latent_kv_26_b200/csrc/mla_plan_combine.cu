@@ -135,6 +135,62 @@ __global__ void __launch_bounds__(256) mla_combine_kernel(CombineArgs a) {
   if (lane == 0) a.lse[row] = m[0] + logf(sum[0]);
 }
 
+// Merge of `parts` results of the same rows computed over disjoint token
+// sets (one per context-parallel shard): one warp per row, lane l holding
+// columns [8l, 8l + 8) and [256 + 8l, 256 + 8l + 8).
+// lse = M + ln sum_i exp(lse_i - M), out = sum_i exp(lse_i - lse) * out_i;
+// parts with lse_i = -inf weigh nothing; all empty: out = 0, lse = -inf.
+__global__ void __launch_bounds__(256) mla_merge_kernel(MergeArgs a) {
+  const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= a.rows) return;
+  float m = -INFINITY;
+  for (int i = 0; i < a.parts; ++i) m = fmaxf(m, a.part_lse[(size_t)i * a.rows + row]);
+  float acc[16];
+#pragma unroll
+  for (int j = 0; j < 16; ++j) acc[j] = 0.f;
+  float sum = 0.f;
+  if (m != -INFINITY) {
+    for (int i = 0; i < a.parts; ++i) {
+      const float l = a.part_lse[(size_t)i * a.rows + row];
+      if (l == -INFINITY) continue;
+      const float e = expf(l - m);
+      sum += e;
+      const uint4* src = reinterpret_cast<const uint4*>(a.part_out + ((size_t)i * a.rows + row) * kDLatent);
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const uint4 v = src[lane + 32 * h];
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[u]));
+          acc[8 * h + 2 * u] += e * f.x;
+          acc[8 * h + 2 * u + 1] += e * f.y;
+        }
+      }
+    }
+  }
+  const float inv = sum > 0.f ? 1.f / sum : 0.f;
+  uint4* dst = reinterpret_cast<uint4*>(a.out + (size_t)row * kDLatent);
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    uint32_t w[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      __nv_bfloat162 b = __floats2bfloat162_rn(acc[8 * h + 2 * u] * inv, acc[8 * h + 2 * u + 1] * inv);
+      w[u] = *reinterpret_cast<uint32_t*>(&b);
+    }
+    dst[lane + 32 * h] = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+  if (lane == 0) a.lse[row] = sum > 0.f ? m + logf(sum) : -INFINITY;
+}
+
+cudaError_t launch_merge(const MergeArgs& args, cudaStream_t stream) {
+  const long long blocks = (args.rows + 7) / 8;
+  mla_merge_kernel<<<(unsigned)blocks, 256, 0, stream>>>(args);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_plan(const PlanArgs& args, cudaStream_t stream) {
   mla_plan_kernel<<<1, 1024, 0, stream>>>(args);
   return cudaGetLastError();
