@@ -62,5 +62,6 @@ from .decode import (  # noqa: F401
 )
 from .plan import split_plan  # noqa: F401
 from .cache_insert import rms_norm, rope_pairs, cache_insert  # noqa: F401,E402
-from .fp8_cache import e4m3_round, quantize_rows, dequantize_rows, fp8_roundtrip_cache  # noqa: F401,E402
+from .fp8_cache import (e4m3_round, quantize_rows, dequantize_rows, fp8_roundtrip_cache, unpack_rows,  # noqa: F401,E402
+                        dequantize_cache)
 from .indexer import index_scores, topk_positions  # noqa: F401,E402

@@ -21,6 +21,10 @@ Readings where the pages are silent:
   kernel would: ``s`` is the float32 quotient ``amax / 448`` and ``x / s`` the
   float32 (IEEE, correctly rounded) quotient; only then is the e4m3 rounding
   applied. The product ``code * s`` is rounded to float32 before bf16.
+* Row layout in memory (the pages print none): one cached token is 656 bytes,
+  ``[0, 512)`` the e4m3 codes of the latent in column order, ``[512, 640)``
+  the 64 rope values as bf16 (little-endian), ``[640, 644)`` the float32
+  scale, ``[644, 656)`` zero (rows stay 16-byte aligned); a page is 64 rows.
 """
 
 from __future__ import annotations
@@ -28,6 +32,9 @@ from __future__ import annotations
 import torch
 
 D_LATENT = 512
+D_ROPE = 64
+ROW_BYTES = 656          # e4m3 codes 512 | bf16 rope 128 | f32 scale 4 | zero 12
+ROPE_OFF, SCALE_OFF = 512, 640
 E4M3_MAX = 448.0
 E4M3_MIN_NORMAL_EXP = -6   # smallest normal 2^-6; subnormal spacing 2^-9
 E4M3_MANT_BITS = 3
@@ -69,4 +76,25 @@ def fp8_roundtrip_cache(cache: torch.Tensor) -> torch.Tensor:
     codes, scale = quantize_rows(cache[..., :D_LATENT])
     out = cache.clone()
     out[..., :D_LATENT] = dequantize_rows(codes, scale).to(cache.dtype)
+    return out
+
+
+def unpack_rows(raw: torch.Tensor):
+    """Raw fp8-cache rows ``[..., 656]`` (uint8) -> (codes as float64 e4m3
+    values [..., 512], float32 scales [...], bf16 rope [..., 64])."""
+    raw = raw.contiguous()
+    codes = raw[..., :D_LATENT].contiguous().view(torch.float8_e4m3fn).to(torch.float64)
+    rope = raw[..., ROPE_OFF:SCALE_OFF].contiguous().view(torch.bfloat16)
+    scale = raw[..., SCALE_OFF:SCALE_OFF + 4].contiguous().view(torch.float32)[..., 0]
+    return codes, scale, rope
+
+
+def dequantize_cache(raw: torch.Tensor) -> torch.Tensor:
+    """An fp8 cache ``[pages, 64, 656]`` (uint8) as the bf16 cache ``[pages, 64,
+    576]`` a decode over it computes with: latent ``bf16(float32(code * s))``,
+    rope unchanged."""
+    codes, scale, rope = unpack_rows(raw)
+    out = torch.empty(raw.shape[:-1] + (D_LATENT + D_ROPE,), dtype=torch.bfloat16)
+    out[..., :D_LATENT] = dequantize_rows(codes, scale).to(torch.bfloat16)
+    out[..., D_LATENT:] = rope
     return out

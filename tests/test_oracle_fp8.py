@@ -103,3 +103,44 @@ def test_decode_over_fp8_cache_single_key_returns_dequantised_latent():
     q = torch.randn(1, 1, 4, 576, generator=gen).to(BF)
     out, _ = oracle.mla_decode(q, rt, torch.zeros(1, 1, dtype=torch.int32), torch.tensor([1], dtype=torch.int32))
     assert torch.equal(out[0, 0], rt[0, 0, :512].to(torch.float64).expand(4, -1))
+
+
+def test_row_layout_unpacks_a_hand_built_row():
+    """A 656-byte row written byte by byte (struct, no tensor views): codes
+    0x38 = 1, 0xB8 = -1, 0x01 = 2^-9 (smallest subnormal), 0x7E = 448 (largest),
+    0x00 = 0; rope bf16 0x3FC0 = 1.5 and 0xC040 = -3; scale float32 2.0;
+    twelve zero bytes. Dequantised: 2, -2, 2^-8, 896, 0; rope unchanged."""
+    import struct
+
+    codes = bytes([0x38, 0xB8, 0x01, 0x7E] + [0x00] * 508)
+    rope = struct.pack("<64H", *([0x3FC0, 0xC040] * 32))
+    row = codes + rope + struct.pack("<f", 2.0) + bytes(12)
+    assert len(row) == f8.ROW_BYTES == 656
+    raw = torch.tensor(list(row), dtype=torch.uint8).view(1, 1, 656)
+    c, s, r = f8.unpack_rows(raw)
+    assert c[0, 0, :5].tolist() == [1.0, -1.0, 2.0 ** -9, 448.0, 0.0]
+    assert float(s[0, 0]) == 2.0
+    assert r[0, 0, :2].to(torch.float64).tolist() == [1.5, -3.0]
+    dq = f8.dequantize_cache(raw)
+    assert dq.shape == (1, 1, 576) and dq.dtype == BF
+    assert dq[0, 0, :5].to(torch.float64).tolist() == [2.0, -2.0, 2.0 ** -8, 896.0, 0.0]
+    assert torch.equal(dq[0, 0, 512:], r[0, 0])
+
+
+def test_dequantize_cache_matches_roundtrip_of_quantised_rows():
+    """Packing quantize_rows' codes and scales into rows by hand and reading
+    them back gives the same cache as fp8_roundtrip_cache."""
+    import struct
+
+    gen = torch.Generator().manual_seed(4)
+    cache = (torch.randn(2, 64, 576, generator=gen) * 2).to(BF)
+    codes, scale = f8.quantize_rows(cache[..., :512])
+    code_bytes = codes.to(torch.float32).to(torch.float8_e4m3fn).view(torch.uint8)
+    rows = []
+    for p in range(2):
+        for t in range(64):
+            rope = cache[p, t, 512:].view(torch.int16).to(torch.int32) & 0xFFFF
+            rows.append(bytes(code_bytes[p, t].tolist()) + struct.pack("<64H", *rope.tolist())
+                        + struct.pack("<f", float(scale[p, t])) + bytes(12))
+    raw = torch.tensor(list(b"".join(rows)), dtype=torch.uint8).view(2, 64, 656)
+    assert torch.equal(f8.dequantize_cache(raw), f8.fp8_roundtrip_cache(cache))
