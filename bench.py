@@ -43,8 +43,9 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # ---------------------------------------------------------------- accounting
 
 
-def accounting(inp: dict) -> dict:
-    """Algorithmic work of one step (no split partials, no re-reads)."""
+def accounting(inp: dict, row_bytes: int = BYTES_PER_TOKEN) -> dict:
+    """Algorithmic work of one step (no split partials, no re-reads); a cached
+    row is ``row_bytes`` (1152 bf16, 656 in the fp8 cache format)."""
     lens = [int(x) for x in inp["seq_lens"]]
     B, Sq, H, topk = inp["batch"], inp["q_len"], inp["heads"], inp["topk"]
     kv_tokens = 0          # distinct cache rows read per sequence
@@ -63,7 +64,7 @@ def accounting(inp: dict) -> dict:
             row_tokens += sum(per_q)
             table_bytes += ((max(per_q) + 63) // 64) * 4
     rows = B * Sq * H
-    bytes_ = kv_tokens * BYTES_PER_TOKEN + rows * 576 * 2 + rows * 512 * 2 + rows * 4 + table_bytes + B * 4
+    bytes_ = kv_tokens * row_bytes + rows * 576 * 2 + rows * 512 * 2 + rows * 4 + table_bytes + B * 4
     flops = row_tokens * H * FLOPS_PER_ROW_TOKEN
     return {"kv_tokens": kv_tokens, "row_tokens": row_tokens, "bytes": bytes_, "flops": flops,
             "h2d_bytes": rows * 576 * 2 + inp["block_table"].numel() * 4 + B * 4 +
@@ -82,11 +83,12 @@ def l2_bytes_of(dev=None) -> int:
     return L2_NOMINAL_BYTES
 
 
-def decode_config(inp: dict, acc: dict, n_gpus: int, l2_bytes: int) -> dict:
+def decode_config(inp: dict, acc: dict, n_gpus: int, l2_bytes: int, cache: str = "bf16") -> dict:
     """The ``config`` object of the decode line; both arms print the same one."""
     w = inp["workload"]
     flush = acc["bytes"] < 2 * l2_bytes
-    return {"workload": f"{w.key} {w.name}", "batch": w.batch, "q_len": w.q_len, "heads": w.heads,
+    name = f"{w.key} {w.name}" + ("" if cache == "bf16" else " fp8-cache (656 B per token)")
+    return {"workload": name, "batch": w.batch, "q_len": w.q_len, "heads": w.heads,
             "kv_len": f"{w.len_lo}..{w.len_hi}" + (f" top{w.topk}" if w.topk else ""),
             "kv_tokens_per_step": acc["kv_tokens"], "bytes_per_step": acc["bytes"],
             "flops_per_step": acc["flops"], "seed": w.seed,
@@ -217,9 +219,13 @@ def oracle_sample(inp: dict, budget_s: float):
     return toks, time.perf_counter() - t0, done
 
 
-def run_reference(args, inp, rank):
+def run_reference(args, inp, rank, row_bytes=BYTES_PER_TOKEN):
     if rank != 0:
         return
+    if inp["cache"].dtype == torch.uint8:
+        import oracle
+
+        inp = dict(inp, cache=oracle.dequantize_cache(inp["cache"]))  # what a decode over the fp8 cache computes with
     torch.set_num_threads(os.cpu_count() or 1)
     # each step: the oracle on a bounded slice (two sequences) of the batch
     per_step = []
@@ -243,7 +249,7 @@ def run_reference(args, inp, rank):
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs_total / max(args.steps, 1),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": decode_config(inp, accounting(inp), args.gpus, l2_bytes_of()),
+        "config": decode_config(inp, accounting(inp, row_bytes), args.gpus, l2_bytes_of(), args.cache),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": torch.get_num_threads(), "kind": "oracle",
                          "sample": "float64 CPU oracle, two whole sequences of the batch per step"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -768,6 +774,8 @@ def main():
                     help="decode: the decode step (default); insert: the latent-cache insert alone; "
                          "absorb: the absorb + un-absorb projections; indexer: fp8 index scores + top-k")
     ap.add_argument("--absorb-tokens", type=int, default=64, help="query tokens for --op absorb")
+    ap.add_argument("--cache", default="bf16", choices=["bf16", "fp8"],
+                    help="decode: the latent cache format (fp8: e4m3 codes + per-token scale, 656 B per token)")
     ap.add_argument("--insert-batch", type=int, default=64)
     ap.add_argument("--insert-tokens", type=int, default=1024, help="new tokens per sequence for --op insert")
     args = ap.parse_args()
@@ -790,9 +798,15 @@ def main():
         return
 
     inp = make_inputs(args.workload)
+    row_bytes = BYTES_PER_TOKEN
+    if args.cache == "fp8":
+        from mla_latent_kv_26_b200.workloads import make_fp8_cache
+
+        inp["cache"] = make_fp8_cache(inp)  # [pages, 64, 656] uint8 replaces the bf16 cache
+        row_bytes = 656
 
     if args.impl == "reference":
-        run_reference(args, inp, rank)
+        run_reference(args, inp, rank, row_bytes)
         return
 
     import torch.distributed as dist
@@ -806,7 +820,7 @@ def main():
 
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
 
-    acc = accounting(inp)
+    acc = accounting(inp, row_bytes)
     g = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
     dec = decoder_for(inp, num_sms=args.num_sms, device=dev)
     stream = torch.cuda.current_stream(dev)
@@ -1000,7 +1014,7 @@ def main():
     else:
         roof = {"bound": "tensor", "achieved": achieved_tf, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                 "frac": achieved_tf / peaks["bf16_tflops"]}
-    roof["traffic"] = profiled_traffic("mla_decode_kernel", args.workload)
+    roof["traffic"] = profiled_traffic("mla_decode_kernel", args.workload + ("" if args.cache == "bf16" else "-fp8"))
     roof["peak_source"] = f"{peak_src} (MEASURED_PEAKS.json burst figures)" if peak_src == "measured" else peak_src
     roof["kernel"] = "mla_decode_kernel"
     roof["roofline_time_us"] = max(t_hbm, t_tc) * 1e6
@@ -1015,8 +1029,8 @@ def main():
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
         "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "bf16", "data": "synthetic",
-        "config": decode_config(inp, acc, world, l2_bytes),
+        "dtype": "bf16" if args.cache == "bf16" else "bf16 (fp8 e4m3 cache expanded to bf16)", "data": "synthetic",
+        "config": decode_config(inp, acc, world, l2_bytes, args.cache),
         "launch": {"decode_workers": dec.num_workers, "ctas_per_worker": 2},
         "roofline": roof,
         "e2e": {"value": job_value(world, acc["kv_tokens"], e2e_ms), "unit": UNIT,
@@ -1034,6 +1048,10 @@ def main():
     }
     if rank == 0 and world == 1:
         torch.set_num_threads(os.cpu_count() or 1)
+        if inp["cache"].dtype == torch.uint8:
+            import oracle
+
+            inp = dict(inp, cache=oracle.dequantize_cache(inp["cache"]))
         toks, secs, nseq = oracle_sample(inp, args.cpu_budget)
         line["cpu_baseline"] = {"value": toks / secs, "unit": UNIT, "cores": torch.get_num_threads(),
                                 "kind": "oracle",

@@ -131,6 +131,25 @@ MLA_API mla_status_t mla_decode(const mla_decode_desc_t* desc, void* plan, const
                         const int32_t* block_table, const int32_t* seq_lens, const int32_t* topk_indices,
                         void* out, float* lse, void* workspace, size_t workspace_bytes, mla_stream_t stream);
 
+/* Steps a2-a7 over an fp8 latent cache: the same attention as mla_decode,
+ * with the cached latent kept as e4m3 codes and a per-token scale (the
+ * deployment format of "DeepSeek-V3.2-Exp unboxing", the Indexer section,
+ * whose reference code imitates it by casting the latent to fp8 and back to
+ * bf16). kv_cache_fp8 is [num_pages, 64, 656] bytes, one 656-byte row per
+ * token: bytes [0, 512) the e4m3 codes of c_kv (column order), [512, 640)
+ * k_pe as 64 bf16, [640, 644) the float32 scale s, [644, 656) zero. The
+ * decode uses c_kv[j] = bf16(float32(code[j] * s)) and k_pe unchanged; every
+ * other argument, the plan, the workspace and mla_combine are those of
+ * mla_decode (plan with mla_decode_plan for the same descriptor). The
+ * kernel loads 656 bytes per token instead of 1152 and expands the codes to
+ * exactly those bf16 values in shared memory before the tensor-core steps.
+ * The rows of a page that a sequence does not reach may hold anything (they
+ * are masked). */
+MLA_API mla_status_t mla_decode_fp8(const mla_decode_desc_t* desc, void* plan, const void* q,
+                                    const void* kv_cache_fp8, const int32_t* block_table, const int32_t* seq_lens,
+                                    const int32_t* topk_indices, void* out, float* lse, void* workspace,
+                                    size_t workspace_bytes, mla_stream_t stream);
+
 /* Step a8: merge split partials by LSE (lse = ln sum_i exp(lse_i),
  * out = sum_i exp(lse_i - lse) out_i) and write empty rows as out = 0,
  * lse = -inf. Must follow mla_decode on the same stream. */
@@ -246,6 +265,18 @@ MLA_API mla_status_t mla_cache_insert(const mla_insert_desc_t* desc, const void*
                                       const float* cos_table, const float* sin_table, const int32_t* seq_ids,
                                       const int32_t* positions, const int32_t* block_table, void* kv_cache,
                                       uint32_t* error_word, mla_stream_t stream);
+
+/* mla_cache_insert writing the fp8 cache format of mla_decode_fp8: the same
+ * bf16 latent bf16(weight * bf16(x / rms)) and rotated k_pe, then per token
+ * s = amax / 448 over the 512 latent values (float32 quotient; s = 1 for an
+ * all-zero latent) and code[j] = e4m3(latent[j] / s) (float32 quotient, round
+ * to nearest even, saturating at 448), written with k_pe, s and the zero
+ * tail into the token's 656-byte row of kv_cache_fp8 [num_pages, 64, 656].
+ * Same descriptor, errors and ordering rules as mla_cache_insert. */
+MLA_API mla_status_t mla_cache_insert_fp8(const mla_insert_desc_t* desc, const void* kv, const void* weight,
+                                          const float* cos_table, const float* sin_table, const int32_t* seq_ids,
+                                          const int32_t* positions, const int32_t* block_table, void* kv_cache_fp8,
+                                          uint32_t* error_word, mla_stream_t stream);
 
 /* ---------------------------------------------------------------------------
  * Absorb / un-absorb: the per-head projections around the latent decode.

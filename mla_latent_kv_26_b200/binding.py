@@ -31,7 +31,8 @@ MLA_DEVERR_POSITION = 0x10
 EXPORTED = (
     "mla_plan_bytes", "mla_workspace_bytes", "mla_num_workers", "mla_decode_plan", "mla_decode",
     "mla_combine", "mla_get_error", "mla_status_string", "mla_decode_noalloc", "mla_cache_insert",
-    "mla_absorb_query", "mla_unabsorb_output", "mla_index_scores", "mla_topk", "mla_merge",
+    "mla_absorb_query", "mla_unabsorb_output", "mla_index_scores", "mla_topk", "mla_merge", "mla_decode_fp8",
+    "mla_cache_insert_fp8",
 )
 
 DEFAULT_SOFTMAX_SCALE = 1.0 / math.sqrt(192.0)
@@ -136,12 +137,13 @@ def make_merge_desc(*, parts: int, rows: int, d_latent: int = 512) -> mla_merge_
     return mla_merge_desc_t(parts, d_latent, rows)
 
 
-def _load() -> ctypes.CDLL:
-    if not os.path.exists(LIB_PATH):
+def load_library(path: str) -> ctypes.CDLL:
+    """A handle on a build of the library at ``path`` with every C signature set."""
+    if not os.path.exists(path):
         raise RuntimeError(
-            f"libmla.so is not built ({LIB_PATH} missing): run `python -m mla_latent_kv_26_b200.build` "
+            f"libmla.so is not built ({path} missing): run `python -m mla_latent_kv_26_b200.build` "
             "(there is no non-CUDA fallback)")
-    lib = ctypes.CDLL(LIB_PATH)
+    lib = ctypes.CDLL(path)
     P = ctypes.c_void_p
     D = ctypes.POINTER(mla_decode_desc_t)
     sig = {
@@ -160,6 +162,8 @@ def _load() -> ctypes.CDLL:
         "mla_index_scores": (ctypes.c_int, [ctypes.POINTER(mla_index_desc_t), P, P, P, P, P, P, P]),
         "mla_topk": (ctypes.c_int, [ctypes.POINTER(mla_topk_desc_t), P, P, P, P]),
         "mla_merge": (ctypes.c_int, [ctypes.POINTER(mla_merge_desc_t), P, P, P, P, P]),
+        "mla_decode_fp8": (ctypes.c_int, [D, P, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]),
+        "mla_cache_insert_fp8": (ctypes.c_int, [ctypes.POINTER(mla_insert_desc_t), P, P, P, P, P, P, P, P, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -168,7 +172,7 @@ def _load() -> ctypes.CDLL:
     return lib
 
 
-_lib = _load()
+_lib = load_library(LIB_PATH)
 
 
 def _ptr(x) -> Optional[int]:
@@ -219,6 +223,22 @@ def mla_decode(desc, plan, q, kv_cache, block_table, seq_lens, topk_indices, out
     return int(_lib.mla_decode(ctypes.byref(desc), _ptr(plan), _ptr(q), _ptr(kv_cache), _ptr(block_table),
                                _ptr(seq_lens), _ptr(topk_indices), _ptr(out), _ptr(lse), _ptr(workspace),
                                int(workspace_bytes), _stream(stream)))
+
+
+def mla_decode_fp8(desc, plan, q, kv_cache_fp8, block_table, seq_lens, topk_indices, out, lse, workspace,
+                   workspace_bytes: int, stream=None) -> int:
+    """mla_decode over an fp8 latent cache [pages, 64, 656] bytes."""
+    return int(_lib.mla_decode_fp8(ctypes.byref(desc), _ptr(plan), _ptr(q), _ptr(kv_cache_fp8), _ptr(block_table),
+                                   _ptr(seq_lens), _ptr(topk_indices), _ptr(out), _ptr(lse), _ptr(workspace),
+                                   int(workspace_bytes), _stream(stream)))
+
+
+def mla_cache_insert_fp8(desc, kv, weight, cos_table, sin_table, seq_ids, positions, block_table, kv_cache_fp8,
+                         error_word=None, stream=None) -> int:
+    """mla_cache_insert writing the fp8 cache format."""
+    return int(_lib.mla_cache_insert_fp8(ctypes.byref(desc), _ptr(kv), _ptr(weight), _ptr(cos_table),
+                                         _ptr(sin_table), _ptr(seq_ids), _ptr(positions), _ptr(block_table),
+                                         _ptr(kv_cache_fp8), _ptr(error_word), _stream(stream)))
 
 
 def mla_combine(desc, plan, workspace, workspace_bytes: int, out, lse, stream=None) -> int:

@@ -37,20 +37,24 @@ def _inputs():
     return files
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+# A test build in which the indexer kernel's pipeline waits give up after
+# 200 ns, so that the bounded-wait error path runs (tests/test_timeout.py).
+SHORT_WAIT_LIB = os.path.join(HERE, "libmla_shortwait.so")
+SHORT_WAIT_DEFINES = ["-DMLA_WAIT_LIMIT_NS=200ull"]
+
+
+def up_to_date(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return False
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return all(os.path.getmtime(f) <= t for f in _inputs())
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and up_to_date():
-        return LIB
+def _compile(lib: str, defines, verbose: bool) -> str:
     cmd = [
         nvcc_path(), *ARCH, "-O3", "-lineinfo", "-std=c++17", "--shared", "-Xcompiler", "-fPIC",
-        "-Xcompiler", "-fvisibility=hidden", "-I", INCLUDE, "-I", CSRC,
-        *[os.path.join(CSRC, f) for f in SOURCES], "-o", LIB + ".tmp",
+        "-Xcompiler", "-fvisibility=hidden", "-I", INCLUDE, "-I", CSRC, *defines,
+        *[os.path.join(CSRC, f) for f in SOURCES], "-o", lib + ".tmp",
     ]
     if verbose:
         cmd.insert(-2, "-Xptxas=-v")
@@ -59,9 +63,24 @@ def build(force: bool = False, verbose: bool = False) -> str:
         raise RuntimeError("nvcc failed:\n" + " ".join(cmd) + "\n" + res.stdout + res.stderr)
     if verbose:
         sys.stderr.write(res.stdout + res.stderr)
-    os.replace(LIB + ".tmp", LIB)
+    os.replace(lib + ".tmp", lib)
+    return lib
+
+
+def build(force: bool = False, verbose: bool = False) -> str:
+    if force or not up_to_date(LIB):
+        _compile(LIB, [], verbose)
     return LIB
+
+
+def build_short_wait(force: bool = False) -> str:
+    """The test build with 200 ns pipeline waits in the indexer kernel."""
+    if force or not up_to_date(SHORT_WAIT_LIB):
+        _compile(SHORT_WAIT_LIB, SHORT_WAIT_DEFINES, False)
+    return SHORT_WAIT_LIB
 
 
 if __name__ == "__main__":
     print(build(force="--force" in sys.argv, verbose="--verbose" in sys.argv))
+    if "--short-wait" in sys.argv:
+        print(build_short_wait(force="--force" in sys.argv))

@@ -11,6 +11,11 @@ constexpr int kPage = 64;        // tokens per cache page
 constexpr int kDLatent = 512;    // c_kv width
 constexpr int kDRope = 64;       // k_pe width
 constexpr int kDQK = 576;        // cached values per token
+// fp8 cache row: e4m3 latent codes [0, 512), bf16 rope [512, 640), f32 scale
+// [640, 644), zero [644, 656).
+constexpr int kF8RowBytes = 656;
+constexpr int kF8RopeOff = 512;
+constexpr int kF8ScaleOff = 640;
 constexpr int kRowsPerTask = 128;  // heads handled by one worker (one TMEM lane each)
 constexpr int kMaxHeads = 128;
 
@@ -52,11 +57,17 @@ struct DecodeArgs {
 // columns] of bf16: boxes of 64 columns (128-byte swizzle) and of 32 columns
 // (64-byte swizzle), each 64 rows high for page tiles and 1 row high for
 // gathers.
+//
+// fp8 cache [num_pages * 64 rows, 656 bytes]: `tile` / `row` are boxes of 128
+// code bytes (no swizzle), the rope boxes 64 bytes wide (64-byte swizzle),
+// and `scale_tile` / `scale_row` 16-byte boxes at the scale's offset.
 struct CacheMaps {
   CUtensorMap tile;
   CUtensorMap row;
   CUtensorMap rope_tile;
   CUtensorMap rope_row;
+  CUtensorMap scale_tile;
+  CUtensorMap scale_row;
 };
 
 struct CombineArgs {

@@ -14,10 +14,10 @@ namespace mla {
 cudaError_t launch_plan(const PlanArgs& args, cudaStream_t stream);
 cudaError_t launch_combine(const CombineArgs& args, int tasks, cudaStream_t stream);
 cudaError_t launch_merge(const MergeArgs& args, cudaStream_t stream);
-const void* decode_kernel_ptr();
-int decode_smem_bytes();
-int decode_threads();
-cudaError_t launch_decode(const CacheMaps& maps, const DecodeArgs& args, int workers,
+const void* decode_kernel_ptr(bool fp8);
+int decode_smem_bytes(bool fp8);
+int decode_threads(bool fp8);
+cudaError_t launch_decode(const CacheMaps& maps, const DecodeArgs& args, int workers, bool fp8,
                           cudaStream_t stream);
 
 namespace {
@@ -45,18 +45,24 @@ bool device_info(DeviceInfo* out) {
     int sms = 0, optin = 0;
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return false;
     if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess) return false;
-    if (optin < decode_smem_bytes()) return false;
-    if (cudaFuncSetAttribute(decode_kernel_ptr(), cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             decode_smem_bytes()) != cudaSuccess)
-      return false;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(2 * (sms / 2), 1, 1);
-    cfg.blockDim = dim3(decode_threads(), 1, 1);
-    cfg.dynamicSmemBytes = decode_smem_bytes();
-    int clusters = 0;
-    if (cudaOccupancyMaxActiveClusters(&clusters, decode_kernel_ptr(), &cfg) != cudaSuccess) {
-      cudaGetLastError();
-      clusters = sms / 2;
+    // both cache formats' kernels: the worker count is the smaller of their co-resident clusters
+    int clusters = sms / 2;
+    for (int f = 0; f < 2; ++f) {
+      const bool fp8 = f == 1;
+      if (optin < decode_smem_bytes(fp8)) return false;
+      if (cudaFuncSetAttribute(decode_kernel_ptr(fp8), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               decode_smem_bytes(fp8)) != cudaSuccess)
+        return false;
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(2 * (sms / 2), 1, 1);
+      cfg.blockDim = dim3(decode_threads(fp8), 1, 1);
+      cfg.dynamicSmemBytes = decode_smem_bytes(fp8);
+      int c = 0;
+      if (cudaOccupancyMaxActiveClusters(&c, decode_kernel_ptr(fp8), &cfg) != cudaSuccess) {
+        cudaGetLastError();
+        c = sms / 2;
+      }
+      if (c < clusters) clusters = c;
     }
     d.sms = sms;
     d.max_clusters = clusters;
@@ -170,9 +176,14 @@ mla_status_t mla_decode_plan(const mla_decode_desc_t* desc, const int32_t* seq_l
   return launch_plan(a, (cudaStream_t)stream) == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
-mla_status_t mla_decode(const mla_decode_desc_t* desc, void* plan, const void* q, const void* kv_cache,
-                        const int32_t* block_table, const int32_t* seq_lens, const int32_t* topk_indices, void* out,
-                        float* lse, void* workspace, size_t workspace_bytes, mla_stream_t stream) {
+}  // extern "C"
+
+namespace mla {
+namespace {
+
+mla_status_t decode_impl(const mla_decode_desc_t* desc, void* plan, const void* q, const void* kv_cache,
+                         const int32_t* block_table, const int32_t* seq_lens, const int32_t* topk_indices, void* out,
+                         float* lse, void* workspace, size_t workspace_bytes, bool fp8, mla_stream_t stream) {
   mla_status_t st = check_desc(desc);
   if (st != MLA_OK) return st;
   if (desc->batch == 0) return MLA_OK;  // nothing to read or write; empty tensors may be NULL
@@ -190,23 +201,39 @@ mla_status_t mla_decode(const mla_decode_desc_t* desc, void* plan, const void* q
 
   PFN_cuTensorMapEncodeTiled_v12000 enc = encoder();
   if (!enc) return MLA_ERR_CUDA;
-  // The cache as a 2-D tensor [num_pages * 64 rows, 576 columns] of bf16:
+  // bf16 cache: a 2-D tensor [num_pages * 64 rows, 576 columns] of bf16:
   // 64-column boxes with 128-byte swizzle (latent columns) and 32-column
-  // boxes with 64-byte swizzle (rope columns), 64 rows (page) or 1 row (gather).
+  // boxes with 64-byte swizzle (rope columns), 64 rows (page) or 1 row
+  // (gather). fp8 cache: [num_pages * 64 rows, 656 bytes] of uint8: boxes of
+  // 128 code bytes (no swizzle), 64 rope bytes (64-byte swizzle) and the
+  // 16 bytes holding the scale.
   CacheMaps maps;
-  cuuint64_t dims[2] = {(cuuint64_t)kDQK, (cuuint64_t)desc->num_pages * kPage};
-  cuuint64_t strides[1] = {(cuuint64_t)kDQK * 2};
+  const bool f8 = fp8;
+  cuuint64_t dims[2] = {(cuuint64_t)(f8 ? kF8RowBytes : kDQK), (cuuint64_t)desc->num_pages * kPage};
+  cuuint64_t strides[1] = {(cuuint64_t)(f8 ? kF8RowBytes : kDQK * 2)};
   cuuint32_t elem[2] = {1, 1};
   auto encode = [&](CUtensorMap* m, cuuint32_t cols, cuuint32_t rows, CUtensorMapSwizzle sw) {
     cuuint32_t box[2] = {cols, rows};
-    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(kv_cache), dims, strides, box, elem,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    return enc(m, f8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+               const_cast<void*>(kv_cache), dims, strides, box, elem, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
   };
-  if (!encode(&maps.tile, 64, kPage, CU_TENSOR_MAP_SWIZZLE_128B) || !encode(&maps.row, 64, 1, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !encode(&maps.rope_tile, 32, kPage, CU_TENSOR_MAP_SWIZZLE_64B) ||
-      !encode(&maps.rope_row, 32, 1, CU_TENSOR_MAP_SWIZZLE_64B))
+  if (!f8) {
+    if (!encode(&maps.tile, 64, kPage, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !encode(&maps.row, 64, 1, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !encode(&maps.rope_tile, 32, kPage, CU_TENSOR_MAP_SWIZZLE_64B) ||
+        !encode(&maps.rope_row, 32, 1, CU_TENSOR_MAP_SWIZZLE_64B))
+      return MLA_ERR_CUDA;
+    maps.scale_tile = maps.tile;
+    maps.scale_row = maps.row;
+  } else if (!encode(&maps.tile, 128, kPage, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+             !encode(&maps.row, 128, 1, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+             !encode(&maps.rope_tile, 64, kPage, CU_TENSOR_MAP_SWIZZLE_64B) ||
+             !encode(&maps.rope_row, 64, 1, CU_TENSOR_MAP_SWIZZLE_64B) ||
+             !encode(&maps.scale_tile, 16, kPage, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+             !encode(&maps.scale_row, 16, 1, CU_TENSOR_MAP_SWIZZLE_NONE)) {
     return MLA_ERR_CUDA;
+  }
 
   const int slots = workers + desc->batch * desc->q_len;
   DecodeArgs a;
@@ -226,7 +253,26 @@ mla_status_t mla_decode(const mla_decode_desc_t* desc, void* plan, const void* q
   a.max_pages_per_seq = desc->max_pages_per_seq;
   a.topk = desc->topk;
   a.scale_log2 = desc->softmax_scale * 1.4426950408889634f;
-  return launch_decode(maps, a, workers, (cudaStream_t)stream) == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+  return launch_decode(maps, a, workers, fp8, (cudaStream_t)stream) == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+}  // namespace
+}  // namespace mla
+
+extern "C" {
+
+mla_status_t mla_decode(const mla_decode_desc_t* desc, void* plan, const void* q, const void* kv_cache,
+                        const int32_t* block_table, const int32_t* seq_lens, const int32_t* topk_indices, void* out,
+                        float* lse, void* workspace, size_t workspace_bytes, mla_stream_t stream) {
+  return decode_impl(desc, plan, q, kv_cache, block_table, seq_lens, topk_indices, out, lse, workspace,
+                     workspace_bytes, false, stream);
+}
+
+mla_status_t mla_decode_fp8(const mla_decode_desc_t* desc, void* plan, const void* q, const void* kv_cache_fp8,
+                            const int32_t* block_table, const int32_t* seq_lens, const int32_t* topk_indices,
+                            void* out, float* lse, void* workspace, size_t workspace_bytes, mla_stream_t stream) {
+  return decode_impl(desc, plan, q, kv_cache_fp8, block_table, seq_lens, topk_indices, out, lse, workspace,
+                     workspace_bytes, true, stream);
 }
 
 mla_status_t mla_combine(const mla_decode_desc_t* desc, void* plan, const void* workspace, size_t workspace_bytes,

@@ -11,7 +11,7 @@
 // contraction with them. The softmax of each head row is owned by one CTA:
 // in every 32-lane TMEM quadrant, CTA r owns lanes [16r, 16r+16). For each
 // tile, a CTA sends the peer the partial scores of the rows the peer owns
-// (16-bit block fixed point, one power-of-two scale per row; 8 KB),
+// (23-bit block fixed point in 3 bytes, one power-of-two scale per row; 12 KB),
 // receives the peer's partials of its own rows, runs the online softmax for
 // its 64 rows, and sends back their P (bf16) together with the per-row
 // rescale factor, running max and running sum (9 KB). Both CTAs then hold the
@@ -63,13 +63,36 @@ constexpr int kVBoxes = 4;              // this CTA's 256 output columns, 4 boxe
 constexpr int kRopeBoxBytes = kPage * 64;  // 64 rows x 32 bf16 (one 64-byte swizzle row each)
 constexpr int kRopeOff = kVBoxes * kBoxBytes;
 constexpr int kStageBytes = kRopeOff + kRopeBoxBytes;
-// Partial-score slot: per quadrant, 32 threads x 6 chunks of 16 B (16 rows x 64 tokens x 3 B).
-// Score slot: per quadrant, 32 threads x 4 chunks of 16 B (16 rows x 64
-// tokens of 16-bit fixed point), then per quadrant 16 row exponents of 4 B.
-constexpr int kXQuadBytes = 32 * 4 * 16;
+// fp8 cache: the CTA's 256 latent columns arrive as e4m3 codes in two boxes
+// of 64 rows x 128 B (no swizzle) in the upper half of the stage's latent
+// region, the rope box as above, and the rows' scales (16 B each) after it;
+// two converter warps then write the bf16 latent boxes in place. Every TMA
+// destination is 128-byte aligned: a page's scales arrive as one box of
+// 64 x 16 B (row r at 16 r), gathered rows four at a time into 128-byte slots
+// (row r at 128 (r / 4) + 16 (r % 4)).
+constexpr int kThreadsF8 = 512;
+constexpr int kF8CodeBoxBytes = kPage * 128;
+constexpr int kF8CodeOff = 2 * kBoxBytes;
+constexpr int kF8ScaleStageOff = kStageBytes;
+constexpr int kF8ScaleBytes = 16 * 128;  // room for the gathered layout
+constexpr int kStageBytesF8 = kStageBytes + kF8ScaleBytes;
+constexpr int kF8LoadBytes = 2 * kF8CodeBoxBytes + kRopeBoxBytes + kPage * 16;
+// Score slot: per quadrant, 32 threads x 6 chunks of 16 B (16 rows x 64
+// tokens of 23-bit fixed point in 3 bytes), then per quadrant 16 row
+// exponents of 4 B.
+// Each quadrant's part (data, then its 16 row exponents) is contiguous, so
+// that one bulk copy per quadrant sends it.
+constexpr int kXChunks = 6;
+constexpr int kXQuadBytes = 32 * kXChunks * 16;
 constexpr int kXExpBytes = 16 * 4;
-constexpr int kXExpOff = 4 * kXQuadBytes;
-constexpr int kXBytes = kXExpOff + 4 * kXExpBytes;
+constexpr int kXQuadStride = kXQuadBytes + kXExpBytes;
+constexpr int kXBytes = 4 * kXQuadStride;
+// One score slot, and one staging buffer from which the sender warps' bulk
+// copies read: the partials of tile k are staged only after the peer has read
+// tile k - 1 out of its slot, which also means the copy of tile k - 1 has
+// finished reading the staging buffer. (A second slot, measured, did not
+// shorten the step.)
+constexpr int kXSlots = 1;
 // P buffer: 128 rows of 64 bf16 (one 128-byte swizzle row each).
 constexpr int kPSlotBytes = 128 * 128;
 constexpr int kPQuadBytes = 16 * 128;    // the 16 rows a CTA owns in one quadrant
@@ -91,17 +114,22 @@ constexpr uint64_t kTimeoutNs = 2000000000ull;
 // swizzle atoms), which holds when the dynamic shared memory base is (checked
 // at run time).
 constexpr int kMiscBytes = 1024;
-constexpr int kSmemBytes =
-    kMiscBytes + kStages * kStageBytes + kPSlots * (kPSlotBytes + kStatBytes) + kXBytes + kQRopeBytes;
-static_assert(kSmemBytes <= 232448, "shared memory budget");
+template <bool kF8>
+constexpr int smem_bytes() {
+  return kMiscBytes + kStages * (kF8 ? kStageBytesF8 : kStageBytes) + kPSlots * (kPSlotBytes + kStatBytes) +
+         (kXSlots + 1) * kXBytes + kQRopeBytes;
+}
+static_assert(smem_bytes<false>() <= 232448 && smem_bytes<true>() <= 232448, "shared memory budget");
+static_assert(kStageBytesF8 % 1024 == 0, "stages hold 128-byte swizzle atoms");
 
 struct Misc {
   uint64_t full[kStages];
   uint64_t empty[kStages];
   uint64_t s_full[2], s_free[2], o_full, o_empty, q_full, mma_done;
   uint64_t p_full[kPSlots], p_free[kPSlots], pm_full[kPSlots];
-  uint64_t x_full, x_empty, x_read;
+  uint64_t x_full[kXSlots], x_empty[kXSlots], x_read[kXSlots];
   uint64_t stage_mask[kStages];
+  uint64_t conv_full[kStages], conv_sync;  // fp8 cache: stage converted; both converter warps hold their codes
   uint32_t tmem_base;
   uint32_t abort_flag;
   uint32_t xdummy[4];  // targets of the peer's 4-byte "slot read" stores
@@ -185,15 +213,18 @@ struct Cursor {
   }
 };
 
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+template <bool kF8>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kF8 ? kThreadsF8 : kThreads, 1)
     mla_decode_kernel(const __grid_constant__ CacheMaps maps, const DecodeArgs a) {
+  constexpr int kSB = kF8 ? kStageBytesF8 : kStageBytes;  // stage stride
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   Misc* misc = reinterpret_cast<Misc*>(smem_raw);
   const uint32_t raw_base = smem_addr(smem_raw);
   const uint32_t stage_base = raw_base + kMiscBytes;
-  const uint32_t pbuf = stage_base + kStages * kStageBytes;  // P buffers (1024-aligned)
-  const uint32_t xbuf = pbuf + kPSlots * kPSlotBytes;         // score slot
-  const uint32_t statbuf = xbuf + kXBytes;                    // stat slots
+  const uint32_t pbuf = stage_base + kStages * kSB;  // P buffers (1024-aligned)
+  const uint32_t xbuf = pbuf + kPSlots * kPSlotBytes;         // score slots
+  const uint32_t xstage = xbuf + kXSlots * kXBytes;           // outgoing partial scores
+  const uint32_t statbuf = xstage + kXBytes;                  // stat slots
   const uint32_t qrope = statbuf + kPSlots * kStatBytes;      // rope columns of Q
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -219,14 +250,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     mbar_init(smem_addr(&misc->o_empty), 8);  // 4 softmax + 4 acceptor warps
     mbar_init(smem_addr(&misc->q_full), 8);   // 4 softmax + 4 sender warps
     mbar_init(smem_addr(&misc->mma_done), 1);
-    mbar_init(smem_addr(&misc->x_full), 1);
-    mbar_init(smem_addr(&misc->x_empty), 1);
-    mbar_init(smem_addr(&misc->x_read), 4);
+    for (int x = 0; x < kXSlots; ++x) {
+      mbar_init(smem_addr(&misc->x_full[x]), 1);
+      mbar_init(smem_addr(&misc->x_empty[x]), 1);
+      mbar_init(smem_addr(&misc->x_read[x]), 4);
+    }
     for (int ps = 0; ps < kPSlots; ++ps) {
       mbar_init(smem_addr(&misc->pm_full[ps]), 1);
       mbar_init(smem_addr(&misc->p_full[ps]), 8);   // 4 softmax + 4 acceptor warps
       mbar_init(smem_addr(&misc->p_free[ps]), 2);   // the PV commits of both CTAs
     }
+    for (int s = 0; s < kStages; ++s) mbar_init(smem_addr(&misc->conv_full[s]), 2);  // the two converter warps
+    mbar_init(smem_addr(&misc->conv_sync), 2);
     misc->abort_flag = 0u;
     fence_mbar_init();
   }
@@ -361,12 +396,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       else if (write_lse) a.lse[qrow] = lse;
     }
   };
-  // The last phase of the score-slot barrier, fed by the peer's 4-byte "slot
-  // read" token for every tile sent, is collected before exit.
+  // The peer's 4-byte "slot read" tokens of the last two tiles sent (the
+  // ones no send waited for) are collected before exit.
   auto drain_x_empty = [&](int tiles, bool expect) {
-    if (tiles > 0) {
-      if (expect) mbar_arrive_expect_tx(smem_addr(&misc->x_empty), 4u);
-      W.wait_cluster_warp(&misc->x_empty, (tiles - 1) & 1);
+    for (int t = max(0, tiles - kXSlots); t < tiles; ++t) {
+      if (expect) mbar_arrive_expect_tx(smem_addr(&misc->x_empty[t % kXSlots]), 4u);
+      W.wait_cluster_warp(&misc->x_empty[t % kXSlots], (t / kXSlots) & 1);
     }
   };
 
@@ -399,13 +434,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             if (lane == 0) {
               misc->stage_mask[s] = mask;
               const uint32_t fb = smem_addr(&misc->full[s]);
-              mbar_arrive_expect_tx(fb, kStageBytes);
               const int row = (ok ? page : 0) * kPage;
-              const uint32_t dst = stage_base + s * kStageBytes;
+              const uint32_t dst = stage_base + s * kSB;
+              if constexpr (kF8) {
+                // codes of this CTA's columns (bytes [256 r, 256 r + 256)), rope, scales
+                mbar_arrive_expect_tx(fb, kF8LoadBytes);
+                tma_load_2d(dst + kF8CodeOff, &maps.tile, vcol0, row, fb);
+                tma_load_2d(dst + kF8CodeOff + kF8CodeBoxBytes, &maps.tile, vcol0 + 128, row, fb);
+                tma_load_2d(dst + kRopeOff, &maps.rope_tile, kF8RopeOff + 64 * (int)crank, row, fb);
+                tma_load_2d(dst + kF8ScaleStageOff, &maps.scale_tile, kF8ScaleOff, row, fb);
+              } else {
+                mbar_arrive_expect_tx(fb, kStageBytes);
 #pragma unroll
-              for (int bx = 0; bx < kVBoxes; ++bx)
-                tma_load_2d(dst + bx * kBoxBytes, &maps.tile, vcol0 + 64 * bx, row, fb);
-              tma_load_2d(dst + kRopeOff, &maps.rope_tile, rcol0, row, fb);
+                for (int bx = 0; bx < kVBoxes; ++bx)
+                  tma_load_2d(dst + bx * kBoxBytes, &maps.tile, vcol0 + 64 * bx, row, fb);
+                tma_load_2d(dst + kRopeOff, &maps.rope_tile, rcol0, row, fb);
+              }
             }
             __syncwarp();
           }
@@ -447,16 +491,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           const uint32_t fb = smem_addr(&misc->full[s]);
           if (lane == 0) {
             misc->stage_mask[s] = mask;
-            mbar_arrive_expect_tx(fb, kStageBytes);
+            mbar_arrive_expect_tx(fb, kF8 ? kF8LoadBytes : kStageBytes);
           }
           __syncwarp();
           if (lane < 16) {
             // lane l gathers tile rows 4l .. 4l+3
-            const uint32_t dst = stage_base + s * kStageBytes;
+            const uint32_t dst = stage_base + s * kSB;
+            if constexpr (kF8) {
+              tma_gather4(dst + kF8CodeOff + lane * 4 * 128, &maps.row, vcol0, r[0], r[1], r[2], r[3], fb);
+              tma_gather4(dst + kF8CodeOff + kF8CodeBoxBytes + lane * 4 * 128, &maps.row, vcol0 + 128, r[0], r[1],
+                          r[2], r[3], fb);
+              tma_gather4(dst + kRopeOff + lane * 4 * 64, &maps.rope_row, kF8RopeOff + 64 * (int)crank, r[0], r[1],
+                          r[2], r[3], fb);
+              tma_gather4(dst + kF8ScaleStageOff + lane * 128, &maps.scale_row, kF8ScaleOff, r[0], r[1], r[2], r[3],
+                          fb);
+            } else {
 #pragma unroll
-            for (int bx = 0; bx < kVBoxes; ++bx)
-              tma_gather4(dst + bx * kBoxBytes + lane * 4 * 128, &maps.row, vcol0 + 64 * bx, r[0], r[1], r[2], r[3], fb);
-            tma_gather4(dst + kRopeOff + lane * 4 * 64, &maps.rope_row, rcol0, r[0], r[1], r[2], r[3], fb);
+              for (int bx = 0; bx < kVBoxes; ++bx)
+                tma_gather4(dst + bx * kBoxBytes + lane * 4 * 128, &maps.row, vcol0 + 64 * bx, r[0], r[1], r[2], r[3],
+                            fb);
+              tma_gather4(dst + kRopeOff + lane * 4 * 64, &maps.rope_row, rcol0, r[0], r[1], r[2], r[3], fb);
+            }
           }
           __syncwarp();
         }
@@ -478,7 +533,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       // at that offset.
       const uint64_t dq = smem_desc_noswz(qrope, kQRopeLbo, kQRopeSbo);
       auto issue_s = [&](int kk) {
-        const uint32_t sb = stage_base + (kk % kStages) * kStageBytes;
+        const uint32_t sb = stage_base + (kk % kStages) * kSB;
         const uint32_t sd = tmem + kTmemS + 64u * (uint32_t)(kk & 1);
         const uint64_t d0 = smem_desc_sw128(sb, 16, 1024);
         const uint64_t dr = smem_desc_sw64(sb + kRopeOff, 512);
@@ -494,7 +549,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       // O (+)= P V for tile kk; releases the P buffer (in both CTAs) and the stage.
       auto issue_pv = [&](int kk, bool first) {
         const int s = kk % kStages;
-        const uint64_t dv = smem_desc_sw128(stage_base + s * kStageBytes, kBoxBytes, 1024);
+        const uint64_t dv = smem_desc_sw128(stage_base + s * kSB, kBoxBytes, 1024);
         const uint64_t dp = smem_desc_sw128(pbuf + (kk & 1) * kPSlotBytes, 16, 1024);
         // K-step u: P advances 32 B along its swizzled rows, V 16 rows (2048 B)
         mma_ss(tmem + kTmemO, dp, dv, idO, first ? 0u : 1u);
@@ -529,7 +584,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           }
           if (ns < n) {
             const int kk = k + ns;
-            if (mbar_test_wait(smem_addr(&misc->full[kk % kStages]), (kk / kStages) & 1) &&
+            // a stage is ready once loaded (and, for the fp8 cache, converted)
+            if (mbar_test_wait(smem_addr(kF8 ? &misc->conv_full[kk % kStages] : &misc->full[kk % kStages]),
+                               (kk / kStages) & 1) &&
                 (kk < 2 || mbar_test_wait(smem_addr(&misc->s_free[kk & 1]), ((kk >> 1) & 1) ^ 1))) {
               tc_fence_after();
               // all 18 MMAs back to back: the tensor pipe overlaps dependent MMAs
@@ -581,9 +638,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const uint32_t pbuf_peer = map_to_rank(pbuf, peer) + pquad;
     const uint32_t stat_peer =
         map_to_rank(statbuf, peer) + (uint32_t)(quad * kStatQuadBytes) + (uint32_t)rl * 16u;
-    const uint32_t xoff = (uint32_t)(quad * kXQuadBytes) + (uint32_t)lane * 16u;
-    const uint32_t xbytes = n_active * (uint32_t)(kXQuadBytes + kXExpBytes);
-    const uint32_t xexp = xbuf + kXExpOff + (uint32_t)(quad * kXExpBytes) + (uint32_t)rl * 4u;
+    const uint32_t xoff = (uint32_t)(quad * kXQuadStride) + (uint32_t)lane * 16u;
+    const uint32_t xbytes = n_active * (uint32_t)kXQuadStride;
+    const uint32_t xexp = xbuf + (uint32_t)(quad * kXQuadStride + kXQuadBytes) + (uint32_t)rl * 4u;
     int k = 0, j = 0;
 
     while (cur.next(task, pg0, pg1, split)) {
@@ -608,30 +665,35 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_addr(&misc->s_free[k & 1]));
-        // the peer's partial scores of these rows
-        if (expect_thread) mbar_arrive_expect_tx(smem_addr(&misc->x_full), xbytes);
-        if (!W.wait_warp(&misc->x_full, k & 1)) goto softmax_done;
+        // the peer's partial scores of these rows, in slot k % 2
+        const uint32_t xslot = (uint32_t)(k % kXSlots) * kXBytes;
+        if (expect_thread) mbar_arrive_expect_tx(smem_addr(&misc->x_full[k % kXSlots]), xbytes);
+        if (!W.wait_warp(&misc->x_full[k % kXSlots], (k / kXSlots) & 1)) goto softmax_done;
         float sc[32];
         {
-          uint32_t w[16];
+          uint32_t w[24];
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            const uint4 v = ld_shared_v4(xbuf + xoff + c * 512);
+          for (int c = 0; c < kXChunks; ++c) {
+            const uint4 v = ld_shared_v4(xbuf + xslot + xoff + c * 512);
             w[4 * c + 0] = v.x;
             w[4 * c + 1] = v.y;
             w[4 * c + 2] = v.z;
             w[4 * c + 3] = v.w;
           }
-          const float inv = fx16_inv(ld_shared_u32(xexp));
-          const float bias = fx16_bias(inv);
+          const float inv = fx23_inv(ld_shared_u32(xexp + xslot));
+          const float bias = fx23_bias(inv);
 #pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            sc[2 * c] = __uint_as_float(own[2 * c]) + fx16_lo(w[c], inv, bias);
-            sc[2 * c + 1] = __uint_as_float(own[2 * c + 1]) + fx16_hi(w[c], inv, bias);
+          for (int c = 0; c < 8; ++c) {
+            float v0, v1, v2, v3;
+            fx23_unpack4(w[3 * c], w[3 * c + 1], w[3 * c + 2], inv, bias, v0, v1, v2, v3);
+            sc[4 * c + 0] = __uint_as_float(own[4 * c + 0]) + v0;
+            sc[4 * c + 1] = __uint_as_float(own[4 * c + 1]) + v1;
+            sc[4 * c + 2] = __uint_as_float(own[4 * c + 2]) + v2;
+            sc[4 * c + 3] = __uint_as_float(own[4 * c + 3]) + v3;
           }
         }
         __syncwarp();
-        if (lane == 0) mbar_arrive(smem_addr(&misc->x_read));
+        if (lane == 0) mbar_arrive(smem_addr(&misc->x_read[k % kXSlots]));
 
         // mask (written by the producer before the stage's full barrier)
         if (!W.wait_warp(&misc->full[s], (k / kStages) & 1)) goto softmax_done;
@@ -703,7 +765,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
         if (mask64 != ~0ull) {
           // masked tokens' V rows may hold anything (even NaN): zero them so 0 * V stays 0
-          const uint32_t sb = stage_base + s * kStageBytes;
+          const uint32_t sb = stage_base + s * kSB;
           for (int e = tid_sm; e < kPage * 32; e += 128) {
             const int r = e >> 5, c = e & 31;
             if (!((mask64 >> r) & 1ull))
@@ -744,20 +806,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   } else if (warp >= 6 && warp <= 9) {
     // ------------------------------------------------------------ sender (rows the peer owns)
     const bool lead = (quad == 0 && lane == 0);  // warp 8, lane 0: expects and relays
-    const uint32_t xfull_peer = map_to_rank(smem_addr(&misc->x_full), peer);
-    const uint32_t xempty_peer = map_to_rank(smem_addr(&misc->x_empty), peer);
-    const uint32_t xbuf_peer = map_to_rank(xbuf, peer) + (uint32_t)(quad * kXQuadBytes) + (uint32_t)lane * 16u;
-    const uint32_t xexp_peer = map_to_rank(xbuf, peer) + kXExpOff + (uint32_t)(quad * kXExpBytes) + (uint32_t)rl * 4u;
+    // peer addresses of slot 0; slot 1 follows at the same stride as here
+    const uint32_t xfull_peer = map_to_rank(smem_addr(&misc->x_full[0]), peer);
+    const uint32_t xempty_peer = map_to_rank(smem_addr(&misc->x_empty[0]), peer);
+    const uint32_t xquad_peer = map_to_rank(xbuf, peer) + (uint32_t)(quad * kXQuadStride);
+    const uint32_t xquad_stage = xstage + (uint32_t)(quad * kXQuadStride);
     const uint32_t xdummy_peer = map_to_rank(smem_addr(&misc->xdummy[quad]), peer);
     int k = 0;
     bool ok = true;
 
-    // This CTA's softmax warps have read the score slot for tile kk: tell the
-    // peer (their arrives released the reads; this wait acquires them).
+    // This CTA's softmax warps have read score slot kk % 2 for tile kk: tell
+    // the peer (their arrives released the reads; this wait acquires them).
     auto relay_read = [&](int kk) -> bool {
       if (quad != 0) return true;
-      if (!W.wait_warp(&misc->x_read, kk & 1)) return false;
-      if (lane == 0) st_async_b32(xdummy_peer, (uint32_t)kk, xempty_peer);
+      if (!W.wait_warp(&misc->x_read[kk % kXSlots], (kk / kXSlots) & 1)) return false;
+      if (lane == 0) st_async_b32(xdummy_peer, (uint32_t)kk, xempty_peer + 8u * (uint32_t)(kk % kXSlots));
       return true;
     };
     // Partial scores of tile kk for the rows the peer owns -> the peer's slot.
@@ -775,7 +838,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_addr(&misc->s_free[kk & 1]));
-      // 16-bit fixed point with the row's exponent; masked tokens (any value,
+      // 23-bit fixed point with the row's exponent; masked tokens (any value,
       // even NaN) neither set the scale nor matter after the receiver masks them
       const int s = kk % kStages;
       if (!W.wait_warp(&misc->full[s], (kk / kStages) & 1)) return false;
@@ -785,19 +848,31 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       for (int c = 0; c < 32; ++c)
         if ((msk >> c) & 1u) amax = fmaxf(amax, fabsf(__uint_as_float(sr[c])));
       amax = fmaxf(amax, __shfl_xor_sync(~0u, amax, 16));
-      const uint32_t ex = fx16_exponent(amax);
-      const float mult = fx16_mult(ex);
-      uint32_t w[16];
+      const uint32_t ex = fx23_exponent(amax);
+      const float mult = fx23_mult(ex);
+      uint32_t w[24];
 #pragma unroll
-      for (int c = 0; c < 16; ++c) w[c] = fx16_pack2(__uint_as_float(sr[2 * c]), __uint_as_float(sr[2 * c + 1]), mult);
-      // the peer's softmax warps have read its slot for tile kk - 1
-      if (kk >= 1 && lead) mbar_arrive_expect_tx(smem_addr(&misc->x_empty), 4u);
-      if (!W.wait_cluster_warp(&misc->x_empty, (kk & 1) ^ 1)) return false;
+      for (int c = 0; c < 8; ++c)
+        fx23_pack4(fx23_code(__uint_as_float(sr[4 * c]), mult), fx23_code(__uint_as_float(sr[4 * c + 1]), mult),
+                   fx23_code(__uint_as_float(sr[4 * c + 2]), mult), fx23_code(__uint_as_float(sr[4 * c + 3]), mult),
+                   w[3 * c], w[3 * c + 1], w[3 * c + 2]);
+      // the peer's softmax warps have read its slot for tile kk - kXSlots (so
+      // that copy has also finished reading this CTA's staging buffer)
+      const int xs = kk % kXSlots;
+      if (kk >= kXSlots && lead) mbar_arrive_expect_tx(smem_addr(&misc->x_empty[xs]), 4u);
+      if (!W.wait_cluster_warp(&misc->x_empty[xs], ((kk / kXSlots) & 1) ^ 1)) return false;
       if (quad_active) {
+        // stage this quadrant's part, then one bulk copy into the peer's slot
 #pragma unroll
-        for (int c = 0; c < 4; ++c)
-          st_async_v4(xbuf_peer + c * 512, w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3], xfull_peer);
-        if (th == 0) st_async_b32(xexp_peer, ex, xfull_peer);
+        for (int c = 0; c < kXChunks; ++c)
+          st_shared_v4(xquad_stage + (uint32_t)(c * 512) + (uint32_t)lane * 16u,
+                       make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]));
+        if (th == 0) st_shared_u32(xquad_stage + (uint32_t)kXQuadBytes + (uint32_t)rl * 4u, ex);
+        fence_proxy_async_smem();  // read by the bulk copy
+        __syncwarp();
+        if (lane == 0)
+          bulk_copy_to_cta(xquad_peer + (uint32_t)xs * kXBytes, xquad_stage, (uint32_t)kXQuadStride,
+                           xfull_peer + 8u * (uint32_t)xs);
       }
       return true;
     };
@@ -813,7 +888,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     // the peer relays "slot read" for every score tile sent; collect the last one before exit
     if (ok) drain_x_empty(k, lead);
     __syncwarp();
-  } else if (warp >= 10) {
+  } else if (warp >= 10 && warp < 14) {
     // ------------------------------------------------------------ acceptor (rows the peer owns)
     const bool lead = (quad == 0 && lane == 0);  // warp 12, lane 0: expects the P messages
     const uint32_t pmbytes = n_active * (uint32_t)(kPQuadBytes + kStatQuadBytes);
@@ -866,6 +941,57 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     __syncwarp();
   }
 
+  if constexpr (kF8) {
+    if (warp >= 14) {
+      // ---------------------------------------------------------- converters (fp8 cache)
+      // Thread ct (0..63) converts 16 chunks of 16 codes per tile: chunk id =
+      // 64 u + ct is row id / 16, columns 16 (id % 16) .. + 15 of this CTA's
+      // 256. All codes are read into registers first: the bf16 boxes written
+      // afterwards cover the codes' bytes.
+      const int ct = (warp - 14) * 32 + lane;
+      int k = 0;
+      bool ok = true;
+      while (ok && cur.next(task, pg0, pg1, split)) {
+        for (int i = pg0; i < pg1; ++i, ++k) {
+          const int s = k % kStages;
+          if (!W.wait_warp(&misc->full[s], (k / kStages) & 1)) {
+            ok = false;
+            break;
+          }
+          const uint32_t sb = stage_base + s * kSB;
+          uint4 cw[16];
+#pragma unroll
+          for (int u = 0; u < 16; ++u) {
+            const int id = 64 * u + ct, row = id >> 4, qc = id & 15;
+            cw[u] = ld_shared_v4(sb + kF8CodeOff + (qc >> 3) * kF8CodeBoxBytes + row * 128 + (qc & 7) * 16);
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(smem_addr(&misc->conv_sync));
+          if (!W.wait_warp(&misc->conv_sync, k & 1)) {
+            ok = false;
+            break;
+          }
+#pragma unroll
+#pragma unroll
+          for (int u = 0; u < 16; ++u) {
+            const int id = 64 * u + ct, row = id >> 4, qc = id & 15;
+            const uint32_t soff = a.topk > 0 ? (uint32_t)((row >> 2) * 128 + (row & 3) * 16) : (uint32_t)(row * 16);
+            const float sc = __uint_as_float(ld_shared_u32(sb + kF8ScaleStageOff + soff));
+            // latent box qc / 4, columns 16 (qc % 4) .. + 15 of it: 16-byte chunks 2 (qc % 4) and + 1
+            const uint32_t box = sb + (uint32_t)((qc >> 2) * kBoxBytes + row * 128);
+            const uint32_t c0 = (uint32_t)(2 * (qc & 3)), sw = (uint32_t)(row & 7);
+            st_shared_v4(box + ((c0 ^ sw) << 4), dequant8_e4m3(cw[u].x, cw[u].y, sc));
+            st_shared_v4(box + (((c0 + 1u) ^ sw) << 4), dequant8_e4m3(cw[u].z, cw[u].w, sc));
+          }
+          fence_proxy_async_smem();  // read by the tensor core
+          __syncwarp();
+          if (lane == 0) mbar_arrive(smem_addr(&misc->conv_full[s]));
+        }
+      }
+      __syncwarp();
+    }
+  }
+
   // ------------------------------------------------------------ teardown
   tc_fence_before();
   cluster_sync();  // no remote access to this CTA's shared memory after this point
@@ -878,13 +1004,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 }  // namespace dec
 
 // Host-side handles (used by mla_api.cu).
-const void* decode_kernel_ptr() { return reinterpret_cast<const void*>(&dec::mla_decode_kernel); }
-int decode_smem_bytes() { return dec::kSmemBytes; }
-int decode_threads() { return dec::kThreads; }
+const void* decode_kernel_ptr(bool fp8) {
+  return fp8 ? reinterpret_cast<const void*>(&dec::mla_decode_kernel<true>)
+             : reinterpret_cast<const void*>(&dec::mla_decode_kernel<false>);
+}
+int decode_smem_bytes(bool fp8) { return fp8 ? dec::smem_bytes<true>() : dec::smem_bytes<false>(); }
+int decode_threads(bool fp8) { return fp8 ? dec::kThreadsF8 : dec::kThreads; }
 
-cudaError_t launch_decode(const CacheMaps& maps, const DecodeArgs& args, int workers,
+cudaError_t launch_decode(const CacheMaps& maps, const DecodeArgs& args, int workers, bool fp8,
                           cudaStream_t stream) {
-  dec::mla_decode_kernel<<<2 * workers, dec::kThreads, dec::kSmemBytes, stream>>>(maps, args);
+  if (fp8)
+    dec::mla_decode_kernel<true><<<2 * workers, dec::kThreadsF8, dec::smem_bytes<true>(), stream>>>(maps, args);
+  else
+    dec::mla_decode_kernel<false><<<2 * workers, dec::kThreads, dec::smem_bytes<false>(), stream>>>(maps, args);
   return cudaGetLastError();
 }
 

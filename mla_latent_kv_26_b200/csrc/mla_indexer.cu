@@ -95,7 +95,15 @@ constexpr int kMaxN = 256;                 // MMA N: query group x heads
 constexpr int kQBytes = kMaxN * kDim;      // 32 KB
 constexpr int kSmem = 1024 + kStages * kTileBytes + 2 * kQBytes;
 constexpr uint32_t kTmemCols = 2 * kMaxN;
-constexpr uint64_t kTimeoutNs = 2000000000ull;
+// A pipeline wait gives up after MLA_WAIT_LIMIT_NS (2 s: only a broken
+// device gets there; a test build sets a few hundred nanoseconds to make the
+// waits run out). The waits that let copies and MMAs in flight finish before
+// the CTA exits keep the 2 s limit in every build.
+#ifndef MLA_WAIT_LIMIT_NS
+#define MLA_WAIT_LIMIT_NS 2000000000ull
+#endif
+constexpr uint64_t kTimeoutNs = MLA_WAIT_LIMIT_NS;
+constexpr uint64_t kDrainNs = 2000000000ull;
 constexpr uint32_t kErrTimeoutBit = 0x8u;
 
 struct Args {
@@ -136,16 +144,40 @@ struct Waiter {
     const uint32_t a = smem_addr(bar);
     if (mbar_try_wait(a, parity)) return true;
     const uint64_t t0 = global_timer_ns();
+    const uint64_t limit = drain ? kDrainNs : kTimeoutNs;
     while (true) {
       if (mbar_try_wait(a, parity)) return true;
       if (!drain && aborted()) return false;
-      if (global_timer_ns() - t0 > kTimeoutNs) {
+      if (global_timer_ns() - t0 > limit) {
         fail();
         return false;
       }
     }
   }
   MLA_DEV bool wait_warp(uint64_t* bar, uint32_t parity) { return __all_sync(~0u, wait(bar, parity)); }
+};
+
+// Position (sequence, query group, key tile) of work item `it`, advanced one
+// item at a time without divisions.
+struct ItemCursor {
+  int bb, g, j, groups, tiles;
+  MLA_DEV void init(long long it, const Args& a) {
+    groups = a.groups;
+    tiles = a.tiles;
+    j = (int)(it % tiles);
+    const long long bg = it / tiles;
+    g = (int)(bg % groups);
+    bb = (int)(bg / groups);
+  }
+  MLA_DEV void next() {
+    if (++j == tiles) {
+      j = 0;
+      if (++g == groups) {
+        g = 0;
+        ++bb;
+      }
+    }
+  }
 };
 
 __global__ void __launch_bounds__(kThreads, 1) mla_index_kernel(const __grid_constant__ Maps maps, const Args a) {
@@ -187,30 +219,26 @@ __global__ void __launch_bounds__(kThreads, 1) mla_index_kernel(const __grid_con
 
   const long long i0 = (long long)blockIdx.x * a.per_cta;
   const long long i1 = min(i0 + a.per_cta, a.items);
-  const long long per_seq = (long long)a.groups * a.tiles;
+  ItemCursor cur;
+  cur.init(i0, a);
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     int k = 0, nq = 0;  // key tiles and query groups whose loads were issued
-    long long prev_bg = -1;
     if (lane == 0) {
-      for (long long it = i0; it < i1; ++it) {
-        const long long bg = it / a.tiles;  // sequence * groups + group
-        const int j = (int)(it % a.tiles);
-        const int bb = (int)(it / per_seq);
-        if (bg != prev_bg) {
-          prev_bg = bg;
+      for (long long it = i0; it < i1; ++it, cur.next()) {
+        if (it == i0 || cur.j == 0) {  // a new query group
           const int qb = nq & 1;
           if (!W.wait(&bars.q_empty[qb], ((nq >> 1) & 1) ^ 1)) break;
-          const int g = (int)(bg % a.groups);
           mbar_arrive_expect_tx(smem_addr(&bars.q_full[qb]), (uint32_t)(a.N * kDim));
-          tma_load_2d(qbuf + qb * kQBytes, &maps.q, 0, (bb * a.m + g * a.G) * a.h, smem_addr(&bars.q_full[qb]));
+          tma_load_2d(qbuf + qb * kQBytes, &maps.q, 0, (cur.bb * a.m + cur.g * a.G) * a.h,
+                      smem_addr(&bars.q_full[qb]));
           ++nq;
         }
         const int s = k % kStages;
         if (!W.wait(&bars.empty[s], ((k / kStages) & 1) ^ 1)) break;
         mbar_arrive_expect_tx(smem_addr(&bars.full[s]), kTileBytes);
-        tma_load_2d(ring + s * kTileBytes, &maps.k, 0, bb * a.n + j * kKeys, smem_addr(&bars.full[s]));
+        tma_load_2d(ring + s * kTileBytes, &maps.k, 0, cur.bb * a.n + cur.j * kKeys, smem_addr(&bars.full[s]));
         ++k;
       }
       // every issued copy lands before the CTA can exit
@@ -223,12 +251,9 @@ __global__ void __launch_bounds__(kThreads, 1) mla_index_kernel(const __grid_con
     if (lane == 0) {
       const uint32_t idesc = idesc_e4m3_f32(kKeys, a.N);
       int k = 0, qi = -1;
-      long long prev_bg = -1;
-      for (long long it = i0; it < i1; ++it) {
-        const long long bg = it / a.tiles;
-        if (bg != prev_bg) {
+      for (long long it = i0; it < i1; ++it, cur.next()) {
+        if (it == i0 || cur.j == 0) {  // a new query group
           if (qi >= 0) mma_commit(smem_addr(&bars.q_empty[qi & 1]));  // the old group's MMAs are issued
-          prev_bg = bg;
           ++qi;
           if (!W.wait(&bars.q_full[qi & 1], (qi >> 1) & 1)) break;
         }
@@ -256,21 +281,28 @@ __global__ void __launch_bounds__(kThreads, 1) mla_index_kernel(const __grid_con
     const int row = quad * 32 + lane;  // key within the tile = TMEM lane
     const uint32_t lanes = tmem + ((uint32_t)(quad * 32) << 16);
     int k = 0;
+    // the key scale of the next item is loaded while this one is computed
+    auto key_scale = [&](const ItemCursor& c) -> float {
+      const int t = c.j * kKeys + row;
+      return t < a.n ? __ldg(a.k_s + (size_t)c.bb * a.n + t) : 0.f;
+    };
+    float ks_next = i0 < i1 ? key_scale(cur) : 0.f;
     for (long long it = i0; it < i1; ++it, ++k) {
       const int tb = k & 1;
+      const ItemCursor c = cur;
+      const float ks = ks_next;
+      cur.next();
+      if (it + 1 < i1) ks_next = key_scale(cur);
       if (!W.wait_warp(&bars.t_full[tb], (k >> 1) & 1)) break;
       tc_fence_after();
-      const int bb = (int)(it / per_seq);
-      const int g = (int)((it / a.tiles) % a.groups);
-      const int j = (int)(it % a.tiles);
-      const int t = j * kKeys + row;
+      const int bb = c.bb, g = c.g;
+      const int t = c.j * kKeys + row;
       const bool valid = t < a.n;
-      const float ks = valid ? __ldg(a.k_s + (size_t)bb * a.n + t) : 0.f;
       const int nq = min(a.G, a.m - g * a.G);
       for (int qj = 0; qj < nq; ++qj) {
         const int mq = g * a.G + qj;
         const float4* w4 = reinterpret_cast<const float4*>(a.q_s + ((size_t)bb * a.m + mq) * a.h);
-        float acc = 0.f;
+        float acc4[4] = {0.f, 0.f, 0.f, 0.f};  // four independent chains over the heads
         for (int c0 = 0; c0 < a.h; c0 += 64) {
           const int nc = min(4, (a.h - c0) >> 4);  // 16-column loads in this round (h is a multiple of 16)
           uint32_t v[4][16];
@@ -284,15 +316,15 @@ __global__ void __launch_bounds__(kThreads, 1) mla_index_kernel(const __grid_con
 #pragma unroll
               for (int e = 0; e < 16; e += 4) {
                 const float4 w = __ldg(w4 + ((c0 + 16 * c + e) >> 2));
-                acc = fmaf(w.x, fmaxf(__uint_as_float(v[c][e + 0]), 0.f), acc);
-                acc = fmaf(w.y, fmaxf(__uint_as_float(v[c][e + 1]), 0.f), acc);
-                acc = fmaf(w.z, fmaxf(__uint_as_float(v[c][e + 2]), 0.f), acc);
-                acc = fmaf(w.w, fmaxf(__uint_as_float(v[c][e + 3]), 0.f), acc);
+                acc4[0] = fmaf(w.x, fmaxf(__uint_as_float(v[c][e + 0]), 0.f), acc4[0]);
+                acc4[1] = fmaf(w.y, fmaxf(__uint_as_float(v[c][e + 1]), 0.f), acc4[1]);
+                acc4[2] = fmaf(w.z, fmaxf(__uint_as_float(v[c][e + 2]), 0.f), acc4[2]);
+                acc4[3] = fmaf(w.w, fmaxf(__uint_as_float(v[c][e + 3]), 0.f), acc4[3]);
               }
             }
           }
         }
-        if (valid) a.o[((size_t)bb * a.m + mq) * a.n + t] = acc * ks;
+        if (valid) a.o[((size_t)bb * a.m + mq) * a.n + t] = ((acc4[0] + acc4[1]) + (acc4[2] + acc4[3])) * ks;
       }
       tc_fence_before();
       __syncwarp();
@@ -356,13 +388,19 @@ MLA_DEV uint32_t block_exclusive_scan(uint32_t v, uint32_t* warp_tot, uint32_t* 
   return before;
 }
 
+// Four 8-bit radix digits, most significant first. Each warp counts into its
+// own 256-bin histogram (the first digits of real scores fall in few bins,
+// and one shared histogram would serialise the whole block on them); the
+// warps' histograms are summed per CTA, then across the cluster.
 __global__ void __launch_bounds__(kTopkThreads, 1) mla_topk_kernel(const TopkArgs a) {
   extern __shared__ __align__(16) uint32_t keys[];
-  __shared__ uint32_t hist[2][256];
+  __shared__ uint32_t whist[32][256];  // per-warp histograms
+  __shared__ uint32_t hist[2][256];    // this CTA's sums, read by the cluster (double-buffered by pass)
   __shared__ uint32_t warp_tot[32];
   __shared__ uint32_t counts[2];  // this CTA's keys above the threshold, keys equal to it
   __shared__ uint32_t pick[2];    // radix pass result: bin, keys in higher bins
-  const int tid = threadIdx.x;
+  __shared__ uint32_t wsum[2][32];  // per warp: keys above, keys equal (selection)
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int C = (int)cluster_nctarank(), c = (int)cluster_ctarank();
   const int row = (int)cluster_id_x();
   const int L = a.lens ? min(max(__ldg(a.lens + row), 0), a.n) : a.n;
@@ -378,14 +416,22 @@ __global__ void __launch_bounds__(kTopkThreads, 1) mla_topk_kernel(const TopkArg
   const bool take_all = K == L;  // uniform over the cluster: every CTA sees the same row
   uint32_t prefix = 0u, mask = 0u, krem = (uint32_t)K;
   if (!take_all) {
+#pragma unroll 1
     for (int p = 0; p < 4; ++p) {
       const int shift = 24 - 8 * p;
-      uint32_t* h = hist[p & 1];
-      if (tid < 256) h[tid] = 0u;
-      __syncthreads();
+      for (int b = lane; b < 256; b += 32) whist[warp][b] = 0u;
+      __syncwarp();
       for (int i = tid; i < cnt; i += kTopkThreads) {
         const uint32_t key = key_at(i);
-        if ((key & mask) == prefix) atomicAdd(&h[(key >> shift) & 255u], 1u);
+        if ((key & mask) == prefix) atomicAdd(&whist[warp][(key >> shift) & 255u], 1u);
+      }
+      __syncthreads();
+      uint32_t* h = hist[p & 1];
+      if (tid < 256) {
+        uint32_t v = 0u;
+#pragma unroll 8
+        for (int w = 0; w < 32; ++w) v += whist[w][tid];
+        h[tid] = v;
       }
       cluster_sync();  // every CTA's histogram of this pass is complete
       // bin b = 255 - tid: an inclusive scan over tid counts the keys in bins >= b
@@ -404,23 +450,40 @@ __global__ void __launch_bounds__(kTopkThreads, 1) mla_topk_kernel(const TopkArg
       krem -= pick[1];
       prefix |= pick[0] << shift;
       mask |= 0xFFu << shift;
-      __syncthreads();  // pick is rewritten by the next pass
+      __syncthreads();  // pick and the warp histograms are rewritten by the next pass
     }
   }
   // prefix is now the k-th largest key T; krem keys equal to T are taken, the
-  // ones at the smallest positions (take_all: every position below L)
+  // ones at the smallest positions (take_all: every position below L).
+  // Selection: warp w walks positions [w * per, (w + 1) * per) in rounds of
+  // 32 consecutive positions (lane order = position order), so prefix counts
+  // come from ballots.
   const uint32_t T = prefix;
-  const int per = (cnt + kTopkThreads - 1) / kTopkThreads;
-  const int b0 = min(tid * per, cnt), b1 = min(b0 + per, cnt);
+  const int per = ((cnt + 32 * 32 - 1) / (32 * 32)) * 32;  // positions per warp, a multiple of 32
+  const int w0 = warp * per, w1 = min(w0 + per, cnt);
   uint32_t gt = 0u, eq = 0u;
-  for (int i = b0; i < b1; ++i) {
-    const uint32_t key = key_at(i);
-    if (take_all || key > T) ++gt;
-    else if (key == T) ++eq;
+  for (int base = w0; base < w1; base += 32) {
+    const int i = base + lane;
+    const uint32_t key = i < w1 ? key_at(i) : 0u;
+    gt += __popc(__ballot_sync(~0u, i < w1 && (take_all || key > T)));
+    eq += __popc(__ballot_sync(~0u, i < w1 && !take_all && key == T));
   }
-  uint32_t g_cta, e_cta;
-  const uint32_t g_pre = block_exclusive_scan(gt, warp_tot, &g_cta);
-  const uint32_t e_pre = block_exclusive_scan(eq, warp_tot, &e_cta);
+  if (lane == 0) {
+    wsum[0][warp] = gt;
+    wsum[1][warp] = eq;
+  }
+  __syncthreads();
+  // this warp's offsets among the CTA's warps (a short serial sum per lane 0)
+  uint32_t g_pre = 0u, e_pre = 0u, g_cta = 0u, e_cta = 0u;
+  for (int w = 0; w < 32; ++w) {
+    const uint32_t gw = wsum[0][w], ew = wsum[1][w];
+    if (w < warp) {
+      g_pre += gw;
+      e_pre += ew;
+    }
+    g_cta += gw;
+    e_cta += ew;
+  }
   if (tid == 0) {
     counts[0] = g_cta;
     counts[1] = e_cta;
@@ -436,18 +499,23 @@ __global__ void __launch_bounds__(kTopkThreads, 1) mla_topk_kernel(const TopkArg
     e_before += e_r;
   }
   const uint32_t take_cta = min(e_cta, krem > e_before ? krem - e_before : 0u);
-  const uint32_t take_me = min(eq, take_cta > e_pre ? take_cta - e_pre : 0u);
-  uint32_t sel_cta;
-  const uint32_t pos = block_exclusive_scan(gt + take_me, warp_tot, &sel_cta);
+  // ties this warp takes: those of the CTA's first take_cta ties that fall in it
+  uint32_t ties_seen = e_pre;                       // CTA ties at positions before this round
+  uint32_t taken_before = min(e_pre, take_cta);     // ties taken by earlier warps
+  uint32_t w = out_base + g_pre + taken_before;     // output slot of this warp's next selection
   int32_t* orow = a.out + (size_t)row * a.k;
-  uint32_t w = out_base + pos, ties = 0u;
-  for (int i = b0; i < b1; ++i) {
-    const uint32_t key = key_at(i);
-    if (take_all || key > T) orow[w++] = lo + i;
-    else if (key == T && ties < take_me) {
-      orow[w++] = lo + i;
-      ++ties;
-    }
+  const uint32_t below = (1u << lane) - 1u;
+  for (int base = w0; base < w1; base += 32) {
+    const int i = base + lane;
+    const uint32_t key = i < w1 ? key_at(i) : 0u;
+    const bool is_gt = i < w1 && (take_all || key > T);
+    const bool is_eq = i < w1 && !take_all && key == T;
+    const uint32_t eqm = __ballot_sync(~0u, is_eq);
+    const bool take_eq = is_eq && ties_seen + __popc(eqm & below) < take_cta;
+    const uint32_t selm = __ballot_sync(~0u, is_gt || take_eq);
+    if (is_gt || take_eq) orow[w + __popc(selm & below)] = lo + i;
+    w += __popc(selm);
+    ties_seen += __popc(eqm);
   }
   if (c == C - 1)
     for (int i = K + tid; i < a.k; i += kTopkThreads) orow[i] = -1;

@@ -76,6 +76,29 @@ MLA_DEV uint4 norm8(uint4 x, uint4 w, float inv) {
 MLA_DEV float sumsq2(uint32_t x) { return bf_lo(x) * bf_lo(x) + bf_hi(x) * bf_hi(x); }
 MLA_DEV float sumsq8(uint4 x) { return sumsq2(x.x) + sumsq2(x.y) + sumsq2(x.z) + sumsq2(x.w); }
 
+// Two floats -> two e4m3 codes (round to nearest even, saturating at +-448),
+// `lo` in the low byte.
+MLA_DEV uint32_t e4m3x2(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+// Eight bf16 values (a uint4) divided by s (IEEE quotients) -> eight e4m3 codes.
+MLA_DEV uint2 codes8(uint4 v, float s) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  uint32_t c[4];
+#pragma unroll
+  for (int u = 0; u < 4; ++u) c[u] = e4m3x2(__fdiv_rn(bf_lo(w[u]), s), __fdiv_rn(bf_hi(w[u]), s));
+  return make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
+}
+MLA_DEV float absmax2(uint32_t v) { return fmaxf(fabsf(bf_lo(v)), fabsf(bf_hi(v))); }
+MLA_DEV float absmax8(uint4 v) { return fmaxf(fmaxf(absmax2(v.x), absmax2(v.y)), fmaxf(absmax2(v.z), absmax2(v.w))); }
+
+// kF8: the row is written in the fp8 cache format (656 bytes: 512 e4m3 codes
+// of the latent divided by its per-token scale amax / 448, the rope as bf16,
+// the float32 scale, 12 zero bytes), from the same bf16 latent values the
+// bf16 format stores.
+template <bool kF8>
 __global__ void __launch_bounds__(kInsertWarps * 32, kInsertBlocksPerSM) mla_insert_kernel(const InsertArgs a) {
   const int lane = threadIdx.x & 31;
   const int warp = blockIdx.x * kInsertWarps + (threadIdx.x >> 5);
@@ -133,11 +156,25 @@ __global__ void __launch_bounds__(kInsertWarps * 32, kInsertBlocksPerSM) mla_ins
       for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
       const float inv = 1.0f / sqrtf(ss * (1.0f / kDLatent) + a.eps);
       const float x0 = bf_lo(xr[u]), x1 = bf_hi(xr[u]);
-      uint4* dst = reinterpret_cast<uint4*>(a.cache + (size_t)row[u] * kDQK);
-      dst[lane] = norm8(xa[u], __ldg(w4 + lane), inv);  // the weight stays in L1
-      dst[32 + lane] = norm8(xb[u], __ldg(w4 + 32 + lane), inv);
-      reinterpret_cast<uint32_t*>(dst + 64)[lane] =
-          ptx::pack_bf16x2(x0 * c[u] - x1 * s[u], x0 * s[u] + x1 * c[u]);
+      const uint4 ya = norm8(xa[u], __ldg(w4 + lane), inv);  // the weight stays in L1
+      const uint4 yb = norm8(xb[u], __ldg(w4 + 32 + lane), inv);
+      const uint32_t rope = ptx::pack_bf16x2(x0 * c[u] - x1 * s[u], x0 * s[u] + x1 * c[u]);
+      if constexpr (!kF8) {
+        uint4* dst = reinterpret_cast<uint4*>(a.cache + (size_t)row[u] * kDQK);
+        dst[lane] = ya;
+        dst[32 + lane] = yb;
+        reinterpret_cast<uint32_t*>(dst + 64)[lane] = rope;
+      } else {
+        float amax = fmaxf(absmax8(ya), absmax8(yb));
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+        const float scale = amax > 0.f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+        uint8_t* dst = reinterpret_cast<uint8_t*>(a.cache) + (size_t)row[u] * kF8RowBytes;
+        *reinterpret_cast<uint2*>(dst + 8 * lane) = codes8(ya, scale);
+        *reinterpret_cast<uint2*>(dst + 256 + 8 * lane) = codes8(yb, scale);
+        *reinterpret_cast<uint32_t*>(dst + kF8RopeOff + 4 * lane) = rope;
+        if (lane == 0) *reinterpret_cast<uint4*>(dst + kF8ScaleOff) = make_uint4(__float_as_uint(scale), 0u, 0u, 0u);
+      }
     }
   }
   if (err && lane == 0 && a.error) atomicOr(a.error, err);
@@ -147,7 +184,7 @@ bool aligned(const void* p, uintptr_t a) { return ((uintptr_t)p & (a - 1)) == 0;
 
 }  // namespace
 
-cudaError_t launch_insert(const InsertArgs& a, cudaStream_t stream) {
+cudaError_t launch_insert(const InsertArgs& a, bool fp8, cudaStream_t stream) {
   if (a.num_tokens == 0) return cudaSuccess;
   int dev = 0, sms = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -156,17 +193,18 @@ cudaError_t launch_insert(const InsertArgs& a, cudaStream_t stream) {
   const int per_block = kInsertWarps * kInsertUnroll;
   const int need = (a.num_tokens + per_block - 1) / per_block;
   const int grid = need < sms * kInsertBlocksPerSM ? need : sms * kInsertBlocksPerSM;
-  mla_insert_kernel<<<grid, kInsertWarps * 32, 0, stream>>>(a);
+  if (fp8) mla_insert_kernel<true><<<grid, kInsertWarps * 32, 0, stream>>>(a);
+  else mla_insert_kernel<false><<<grid, kInsertWarps * 32, 0, stream>>>(a);
   return cudaGetLastError();
 }
 
 }  // namespace mla
 
-extern "C" MLA_API mla_status_t mla_cache_insert(const mla_insert_desc_t* desc, const void* kv, const void* weight,
-                                                 const float* cos_table, const float* sin_table,
-                                                 const int32_t* seq_ids, const int32_t* positions,
-                                                 const int32_t* block_table, void* kv_cache, uint32_t* error_word,
-                                                 mla_stream_t stream) {
+namespace {
+mla_status_t cache_insert(const mla_insert_desc_t* desc, const void* kv, const void* weight, const float* cos_table,
+                          const float* sin_table, const int32_t* seq_ids, const int32_t* positions,
+                          const int32_t* block_table, void* kv_cache, uint32_t* error_word, bool fp8,
+                          mla_stream_t stream) {
   using namespace mla;
   if (!desc) return MLA_ERR_INVALID_ARG;
   if (desc->num_tokens < 0 || desc->batch < 0 || desc->max_pages_per_seq < 1 || desc->num_pages < 1 ||
@@ -198,5 +236,24 @@ extern "C" MLA_API mla_status_t mla_cache_insert(const mla_insert_desc_t* desc, 
   a.num_pages = desc->num_pages;
   a.max_positions = desc->max_positions;
   a.eps = desc->eps;
-  return launch_insert(a, (cudaStream_t)stream) == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+  return launch_insert(a, fp8, (cudaStream_t)stream) == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+}  // namespace
+
+extern "C" MLA_API mla_status_t mla_cache_insert(const mla_insert_desc_t* desc, const void* kv, const void* weight,
+                                                 const float* cos_table, const float* sin_table,
+                                                 const int32_t* seq_ids, const int32_t* positions,
+                                                 const int32_t* block_table, void* kv_cache, uint32_t* error_word,
+                                                 mla_stream_t stream) {
+  return cache_insert(desc, kv, weight, cos_table, sin_table, seq_ids, positions, block_table, kv_cache, error_word,
+                      false, stream);
+}
+
+extern "C" MLA_API mla_status_t mla_cache_insert_fp8(const mla_insert_desc_t* desc, const void* kv,
+                                                     const void* weight, const float* cos_table,
+                                                     const float* sin_table, const int32_t* seq_ids,
+                                                     const int32_t* positions, const int32_t* block_table,
+                                                     void* kv_cache_fp8, uint32_t* error_word, mla_stream_t stream) {
+  return cache_insert(desc, kv, weight, cos_table, sin_table, seq_ids, positions, block_table, kv_cache_fp8,
+                      error_word, true, stream);
 }

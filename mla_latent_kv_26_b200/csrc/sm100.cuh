@@ -1,12 +1,14 @@
 // Thin inline-PTX wrappers for the sm_100a features the decode kernel uses:
 // mbarriers, TMA tile and gather4 loads, cluster/DSMEM access (asynchronous
 // remote stores, bulk copies), tcgen05 (TMEM allocation, MMA, commit,
-// loads/stores, fences), and the 16-bit block fixed-point packing of the
+// loads/stores, fences), and the 23-bit block fixed-point packing of the
 // score exchange. Written from the public PTX ISA.
 #pragma once
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
 #include <stdint.h>
 
 #define MLA_DEV __device__ __forceinline__
@@ -167,6 +169,9 @@ MLA_DEV uint4 ld_shared_v4(uint32_t addr) {
   asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
   return v;
 }
+MLA_DEV void st_shared_u32(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
 MLA_DEV void st_shared_v4(uint32_t addr, uint4 v) {
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
                : "memory");
@@ -215,6 +220,7 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int a_mn_maj
   return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)a_mn_major << 15) | ((uint32_t)b_mn_major << 16) |
          ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
+
 
 // D[tmem] (+)= A[tmem] * B[smem]; issued by one thread.
 MLA_DEV void mma_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc, uint32_t accumulate) {
@@ -298,35 +304,64 @@ MLA_DEV float ex2(float x) {
   return y;
 }
 
-// 16-bit block fixed point (one power-of-two scale per row of 64 values):
-// with E the biased exponent of the row's largest magnitude (at least 15),
-// q = round(x * 2^(141 - E)) lies in [-32767, 32767] and x = q * 2^(E - 141),
-// so the absolute error is at most 2^(E - 142) <= max|x| * 2^-15.
-MLA_DEV uint32_t fx16_exponent(float amax) { return max((__float_as_uint(amax) >> 23) & 0xFFu, 15u); }
-MLA_DEV float fx16_mult(uint32_t e) { return __uint_as_float((268u - e) << 23); }  // 2^(141 - e)
-MLA_DEV float fx16_inv(uint32_t e) { return __uint_as_float((e - 14u) << 23); }    // 2^(e - 141)
-// Two values -> q + 32768 in the low and high halves: the sum with
-// 1.5 * 2^23 + 2^15 has unit spacing, so its low 16 bits are round(x m) + 2^15.
-MLA_DEV uint32_t fx16_pack2(float a, float b, float mult) {
-  constexpr float kMagic = 12615680.0f, kLo = kMagic - 32767.0f, kHi = kMagic + 32767.0f;
-  const float x = fminf(fmaxf(fmaf(a, mult, kMagic), kLo), kHi);
-  const float y = fminf(fmaxf(fmaf(b, mult, kMagic), kLo), kHi);
-  return __byte_perm(__float_as_uint(x), __float_as_uint(y), 0x5410);
+// 23-bit block fixed point (one power-of-two scale per row of 64 values):
+// with E the biased exponent of the row's largest magnitude (at least 22),
+// q = round(x * 2^(148 - E)) lies in [-(2^22 - 1), 2^22 - 1] and
+// x = q * 2^(E - 148), so the absolute error is at most
+// 2^(E - 149) <= max|x| * 2^-22. Four values travel in three 32-bit words.
+MLA_DEV uint32_t fx23_exponent(float amax) { return max((__float_as_uint(amax) >> 23) & 0xFFu, 22u); }
+MLA_DEV float fx23_mult(uint32_t e) { return __uint_as_float((275u - e) << 23); }  // 2^(148 - e)
+MLA_DEV float fx23_inv(uint32_t e) { return __uint_as_float((e - 21u) << 23); }    // 2^(e - 148)
+// x * mult + 1.5 * 2^23 has unit spacing: its low 23 bits are round(x mult) + 2^22
+// (bit 23, the exponent's lowest bit, is 0 over the clamped range).
+MLA_DEV uint32_t fx23_code(float x, float mult) {
+  constexpr float kMagic = 12582912.0f, kLo = kMagic - 4194303.0f, kHi = kMagic + 4194303.0f;
+  return __float_as_uint(fminf(fmaxf(fmaf(x, mult, kMagic), kLo), kHi));
 }
-// q * inv from the low / high half: 2^23 + (q + 2^15) is built by a byte
-// permute, and (2^23 + u) * inv - (2^23 + 2^15) * inv is exact in one FMA.
-MLA_DEV float fx16_bias(float inv) { return -8421376.0f * inv; }
-MLA_DEV float fx16_lo(uint32_t w, float inv, float bias) {
-  return fmaf(__uint_as_float(__byte_perm(w, 0x4B000000u, 0x7410)), inv, bias);
+// Four codes (low three bytes of each) -> three words.
+MLA_DEV void fx23_pack4(uint32_t c0, uint32_t c1, uint32_t c2, uint32_t c3, uint32_t& w0, uint32_t& w1, uint32_t& w2) {
+  w0 = __byte_perm(c0, c1, 0x4210);
+  w1 = __byte_perm(c1, c2, 0x5421);
+  w2 = __byte_perm(c2, c3, 0x6542);
 }
-MLA_DEV float fx16_hi(uint32_t w, float inv, float bias) {
-  return fmaf(__uint_as_float(__byte_perm(w, 0x4B000000u, 0x7432)), inv, bias);
+// q * inv from a 23-bit field u: 2^23 + u is rebuilt as float bits, and
+// (2^23 + u) * inv - (2^23 + 2^22) * inv is exact in one FMA.
+MLA_DEV float fx23_bias(float inv) { return -12582912.0f * inv; }
+MLA_DEV float fx23_val(uint32_t bits24, float inv, float bias) {
+  return fmaf(__uint_as_float((bits24 & 0x00FFFFFFu) | 0x4B000000u), inv, bias);
+}
+// Three words -> four values.
+MLA_DEV void fx23_unpack4(uint32_t w0, uint32_t w1, uint32_t w2, float inv, float bias, float& v0, float& v1,
+                          float& v2, float& v3) {
+  v0 = fx23_val(w0, inv, bias);
+  v1 = fx23_val(__byte_perm(w0, w1, 0x0543), inv, bias);
+  v2 = fx23_val(__byte_perm(w1, w2, 0x0432), inv, bias);
+  v3 = fx23_val(w2 >> 8, inv, bias);
 }
 
 // Two floats -> bf16x2 (round to nearest even), `lo` in the low half.
 MLA_DEV uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// Eight e4m3 codes (two words, lowest byte first) times a float32 scale,
+// each product rounded to float32 and then to bf16: eight bf16 in a uint4.
+// The hardware widens two codes at a time to f16 (exact: every e4m3 value is
+// an f16 normal or zero), f16 -> float32 is exact, the product is one FMUL.
+MLA_DEV uint4 dequant8_e4m3(uint32_t w0, uint32_t w1, float s) {
+  const uint32_t w[2] = {w0, w1};
+  uint32_t o[4];
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      const __nv_fp8x2_storage_t pair = (__nv_fp8x2_storage_t)((w[h] >> (16 * q)) & 0xFFFFu);
+      const float2 f = __half22float2(__half2(__nv_cvt_fp8x2_to_halfraw2(pair, __NV_E4M3)));
+      o[2 * h + q] = pack_bf16x2(__fmul_rn(f.x, s), __fmul_rn(f.y, s));
+    }
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
 }  // namespace ptx

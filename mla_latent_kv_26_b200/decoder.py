@@ -51,17 +51,24 @@ class MlaDecoder:
 
     def decode_step(self, q, kv_cache, block_table, seq_lens, indices: Optional[torch.Tensor] = None,
                     stream=None) -> None:
+        """``kv_cache``: bf16 [pages, 64, 576], or uint8 [pages, 64, 656] for an
+        fp8 latent cache (mla_decode_fp8)."""
         d = self.desc
         self._check("q", q, torch.bfloat16, (d.batch, d.q_len, d.num_heads, 576))
-        self._check("kv_cache", kv_cache, torch.bfloat16, (d.num_pages, 64, 576))
+        fp8 = kv_cache.dtype == torch.uint8
+        if fp8:
+            self._check("kv_cache", kv_cache, torch.uint8, (d.num_pages, 64, 656))
+        else:
+            self._check("kv_cache", kv_cache, torch.bfloat16, (d.num_pages, 64, 576))
         self._check("block_table", block_table, torch.int32, (d.batch, d.max_pages_per_seq))
         self._check("seq_lens", seq_lens, torch.int32, (d.batch,))
         if d.topk > 0:
             self._check("indices", indices, torch.int32, (d.batch, d.q_len, d.topk))
         elif indices is not None:
             raise ValueError("indices given for a dense descriptor")
-        B.check(B.mla_decode(d, self.plan, q, kv_cache, block_table, seq_lens, indices, self.out, self.lse,
-                             self.workspace, self.workspace_bytes, self._stream(stream)), "mla_decode")
+        fn = B.mla_decode_fp8 if fp8 else B.mla_decode
+        B.check(fn(d, self.plan, q, kv_cache, block_table, seq_lens, indices, self.out, self.lse,
+                   self.workspace, self.workspace_bytes, self._stream(stream)), "mla_decode")
 
     def combine_step(self, stream=None) -> None:
         B.check(B.mla_combine(self.desc, self.plan, self.workspace, self.workspace_bytes, self.out, self.lse,
@@ -89,7 +96,8 @@ def cache_insert(kv: torch.Tensor, weight: torch.Tensor, cos: torch.Tensor, sin:
                  positions: torch.Tensor, block_table: torch.Tensor, kv_cache: torch.Tensor, *, eps: float = 1e-6,
                  error_word: Optional[torch.Tensor] = None, stream=None) -> None:
     """kv_norm + RoPE of the new tokens' rows ``kv`` [N, 576], written in place
-    into their rows of ``kv_cache`` [pages, 64, 576] (one library kernel).
+    into their rows of ``kv_cache`` [pages, 64, 576] bf16, or of an fp8 cache
+    [pages, 64, 656] uint8 (mla_cache_insert_fp8), in one library kernel.
     ``error_word``: optional int32 [1] device tensor that collects the
     MLA_DEVERR bits of skipped tokens."""
     dev = kv_cache.device
@@ -97,22 +105,26 @@ def cache_insert(kv: torch.Tensor, weight: torch.Tensor, cos: torch.Tensor, sin:
     want = [("kv", kv, torch.bfloat16, (n, 576)), ("weight", weight, torch.bfloat16, (512,)),
             ("cos", cos, torch.float32, (cos.shape[0], 32)), ("sin", sin, torch.float32, tuple(cos.shape)),
             ("seq_ids", seq_ids, torch.int32, (n,)), ("positions", positions, torch.int32, (n,)),
-            ("block_table", block_table, torch.int32, None), ("kv_cache", kv_cache, torch.bfloat16, None)]
+            ("block_table", block_table, torch.int32, None),
+            ("kv_cache", kv_cache, torch.uint8 if kv_cache.dtype == torch.uint8 else torch.bfloat16, None)]
     for name, t, dtype, shape in want:
         if t.device != dev or t.dtype != dtype or not t.is_contiguous():
             raise ValueError(f"{name}: need a contiguous {dtype} tensor on {dev}")
         if shape is not None and tuple(t.shape) != tuple(shape):
             raise ValueError(f"{name}: shape {tuple(t.shape)} != {tuple(shape)}")
-    if block_table.dim() != 2 or kv_cache.dim() != 3 or tuple(kv_cache.shape[1:]) != (64, 576):
-        raise ValueError("block_table must be [batch, max_pages_per_seq], kv_cache [pages, 64, 576]")
+    fp8 = kv_cache.dtype == torch.uint8
+    if block_table.dim() != 2 or kv_cache.dim() != 3 or tuple(kv_cache.shape[1:]) != (64, 656 if fp8 else 576):
+        raise ValueError("block_table must be [batch, max_pages_per_seq], kv_cache [pages, 64, 576] bf16 "
+                         "or [pages, 64, 656] uint8")
     if error_word is not None and (error_word.device != dev or error_word.dtype != torch.int32):
         raise ValueError("error_word: need an int32 tensor on the cache's device")
     desc = B.make_insert_desc(num_tokens=n, batch=block_table.shape[0], max_pages_per_seq=max(block_table.shape[1], 1),
                               num_pages=kv_cache.shape[0], max_positions=cos.shape[0], eps=eps)
     s = torch.cuda.current_stream(dev) if stream is None else stream
     with torch.cuda.device(dev):
-        B.check(B.mla_cache_insert(desc, kv, weight, cos, sin, seq_ids, positions, block_table, kv_cache, error_word,
-                                   s), "mla_cache_insert")
+        fn = B.mla_cache_insert_fp8 if fp8 else B.mla_cache_insert
+        B.check(fn(desc, kv, weight, cos, sin, seq_ids, positions, block_table, kv_cache, error_word, s),
+                "mla_cache_insert")
 
 
 def _check_tensor(name, t, dtype, shape, dev):

@@ -234,3 +234,53 @@ def indexer_inputs(*, batch: int, q_len: int, heads: int, num_keys: int, seed: i
     k_s = (0.5 + torch.rand(batch, num_keys, generator=g)) / code_std
     return {"q": q, "q_s": q_s, "k": k, "k_s": k_s, "batch": batch, "q_len": q_len, "heads": heads,
             "num_keys": num_keys}
+
+
+FP8_ROW_BYTES = 656  # e4m3 latent codes 512 | bf16 rope 128 | f32 scale 4 | zero 12
+
+
+def make_fp8_cache(inp: dict, *, seed: Optional[int] = None, code_std: float = 64.0,
+                   nan_tail: bool = False) -> torch.Tensor:
+    """An fp8 latent cache ``[num_pages, 64, 656]`` (uint8 rows: 512 e4m3
+    codes, 64 bf16 rope values, a float32 scale, 12 zero bytes) for the page
+    layout of ``inp`` (a dict from :func:`make_inputs`), drawn directly — no
+    quantisation: codes ~ N(0, code_std^2) clipped to the e4m3 range and cast
+    by the library, scales ~ U[0.5, 1.5) * cache_std / code_std, rope ~
+    N(0, cache_std^2) in bf16. Draw order from one generator (seed: the
+    workload's + 1000): codes -> scales -> rope. Pages no sequence owns, and
+    with ``nan_tail`` the unused rows of each sequence's last page, are NaN
+    (codes 0x7F, NaN scale and rope)."""
+    w = inp["workload"]
+    g = torch.Generator().manual_seed((w.seed if seed is None else seed) + 1000)
+    P = inp["num_pages"]
+    raw = torch.zeros(P, PAGE, FP8_ROW_BYTES, dtype=torch.uint8)
+    rows = raw.view(P * PAGE, FP8_ROW_BYTES)
+    n = P * PAGE
+    step = 1 << 14
+    for r0 in range(0, n, step):
+        r1 = min(n, r0 + step)
+        codes = (torch.randn(r1 - r0, D_LATENT, generator=g) * code_std).clamp(-448, 448)
+        rows[r0:r1, :D_LATENT] = codes.to(torch.float8_e4m3fn).view(torch.uint8)
+    scales = (0.5 + torch.rand(n, generator=g)) * (w.cache_std / code_std)
+    rows[:, 640:644] = scales.to(torch.float32).view(torch.uint8).view(n, 4)
+    for r0 in range(0, n, step):
+        r1 = min(n, r0 + step)
+        rope = (torch.randn(r1 - r0, 64, generator=g) * w.cache_std).to(torch.bfloat16)
+        rows[r0:r1, 512:640] = rope.view(torch.uint8).view(r1 - r0, 128)
+
+    def poison(sel):
+        sel[..., :D_LATENT] = 0x7F
+        sel[..., 512:640] = torch.full(sel.shape[:-1] + (64,), float("nan"), dtype=torch.bfloat16).view(
+            torch.uint8).view(sel.shape[:-1] + (128,))
+        sel[..., 640:644] = torch.full(sel.shape[:-1] + (1,), float("nan")).view(torch.uint8).view(
+            sel.shape[:-1] + (4,))
+
+    used = int(sum((int(L) + PAGE - 1) // PAGE for L in inp["seq_lens"].tolist()))
+    if used < P:
+        poison(raw[used:])
+    if nan_tail:
+        bt = inp["block_table"]
+        for b, L in enumerate(inp["seq_lens"].tolist()):
+            if L % PAGE and L > 0:
+                poison(raw[int(bt[b, (L - 1) // PAGE]), L % PAGE:])
+    return raw

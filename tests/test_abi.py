@@ -24,7 +24,8 @@ def _declared():
 
 def test_header_declares_the_boundary():
     assert _declared() == sorted([
-        "mla_absorb_query", "mla_cache_insert", "mla_combine", "mla_decode", "mla_decode_noalloc", "mla_decode_plan",
+        "mla_absorb_query", "mla_cache_insert", "mla_cache_insert_fp8", "mla_combine", "mla_decode", "mla_decode_fp8",
+        "mla_decode_noalloc", "mla_decode_plan",
         "mla_get_error", "mla_index_scores", "mla_merge", "mla_num_workers", "mla_plan_bytes", "mla_status_string",
         "mla_topk", "mla_unabsorb_output", "mla_workspace_bytes"])
 
@@ -288,3 +289,24 @@ def test_merge_bad_arguments_rejected(libmla):
         a[i] += off
         assert libmla.mla_merge(mk(parts=2, rows=4), *a, None) == INV, i
     assert libmla.mla_merge(mk(parts=2, rows=0), None, None, None, None, None) == libmla.MLA_OK
+
+
+def test_fp8_entries_validate_like_their_bf16_counterparts(libmla):
+    """mla_decode_fp8 and mla_cache_insert_fp8 share the argument checks of
+    mla_decode and mla_cache_insert (rejected before any launch)."""
+    for kw, status in [(dict(batch=-1), 1), (dict(d_latent=256), 2), (dict(num_heads=129), 2),
+                       (dict(causal=True, topk=4), 1)]:
+        d = _desc(libmla, **kw)
+        assert libmla.mla_decode_fp8(d, 16, 16, 16, 16, 16, 16, 16, 16, 16, 1 << 30, None) == status
+    d = _desc(libmla)
+    args = [16] * 9
+    for i in range(9):
+        if i == 5:
+            continue
+        a = list(args)
+        a[i] = None
+        assert libmla.mla_decode_fp8(d, *a, 1 << 30, None) == libmla.MLA_ERR_INVALID_ARG, i
+    for kw, status in [(dict(num_tokens=-1), 1), (dict(eps=-1.0), 1), (dict(d_latent=256), 2)]:
+        assert libmla.mla_cache_insert_fp8(_idesc(libmla, **kw), 16, 16, 16, 16, 16, 16, 16, 16, None, None) == status
+    assert libmla.mla_cache_insert_fp8(_idesc(libmla), 16, 16, 16, 16, 16, 16, 16, 24, None, None) == \
+        libmla.MLA_ERR_INVALID_ARG
