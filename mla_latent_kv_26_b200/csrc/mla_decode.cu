@@ -129,7 +129,7 @@ struct Misc {
   uint64_t p_full[kPSlots], p_free[kPSlots], pm_full[kPSlots];
   uint64_t x_full[kXSlots], x_empty[kXSlots], x_read[kXSlots];
   uint64_t stage_mask[kStages];
-  uint64_t conv_full[kStages], conv_sync;  // fp8 cache: stage converted; both converter warps hold their codes
+  uint64_t conv_full[kStages];  // fp8 cache: stage converted to bf16
   uint32_t tmem_base;
   uint32_t abort_flag;
   uint32_t xdummy[4];  // targets of the peer's 4-byte "slot read" stores
@@ -261,7 +261,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kF8 ? kThreadsF8 : k
       mbar_init(smem_addr(&misc->p_free[ps]), 2);   // the PV commits of both CTAs
     }
     for (int s = 0; s < kStages; ++s) mbar_init(smem_addr(&misc->conv_full[s]), 2);  // the two converter warps
-    mbar_init(smem_addr(&misc->conv_sync), 2);
     misc->abort_flag = 0u;
     fence_mbar_init();
   }
@@ -944,11 +943,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kF8 ? kThreadsF8 : k
   if constexpr (kF8) {
     if (warp >= 14) {
       // ---------------------------------------------------------- converters (fp8 cache)
-      // Thread ct (0..63) converts 16 chunks of 16 codes per tile: chunk id =
-      // 64 u + ct is row id / 16, columns 16 (id % 16) .. + 15 of this CTA's
-      // 256. All codes are read into registers first: the bf16 boxes written
-      // afterwards cover the codes' bytes.
-      const int ct = (warp - 14) * 32 + lane;
+      // Thread r (0..63) expands row r of each tile: its 256 codes (code box
+      // 0: columns 0..127, box 1: 128..255, 128 bytes per row) into the four
+      // bf16 boxes (128-byte swizzle). Every output row overlaps only the
+      // same row's codes (box 2 over code box 0, box 3 over code box 1), so
+      // a thread's writes never cover bytes another thread still has to read:
+      // columns 0..191 are converted in place chunk by chunk (their outputs
+      // land on codes the thread has already read), the last 64 codes are
+      // read into registers before box 3 is written. Chunks are taken in an
+      // order rotated by the row, which spreads a warp's accesses over the
+      // shared-memory banks.
+      const int r = (warp - 14) * 32 + lane;
+      const uint32_t sw = (uint32_t)(r & 7);
       int k = 0;
       bool ok = true;
       while (ok && cur.next(task, pg0, pg1, split)) {
@@ -959,30 +965,32 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kF8 ? kThreadsF8 : k
             break;
           }
           const uint32_t sb = stage_base + s * kSB;
-          uint4 cw[16];
-#pragma unroll
-          for (int u = 0; u < 16; ++u) {
-            const int id = 64 * u + ct, row = id >> 4, qc = id & 15;
-            cw[u] = ld_shared_v4(sb + kF8CodeOff + (qc >> 3) * kF8CodeBoxBytes + row * 128 + (qc & 7) * 16);
+          const uint32_t soff = a.topk > 0 ? (uint32_t)((r >> 2) * 128 + (r & 3) * 16) : (uint32_t)(r * 16);
+          const float sc = __uint_as_float(ld_shared_u32(sb + kF8ScaleStageOff + soff));
+          const uint32_t codes = sb + kF8CodeOff + (uint32_t)r * 128u;
+          // 16 codes (columns 16 q .. 16 q + 15) -> two 16-byte chunks of bf16 box q / 4
+          auto put = [&](int q, uint4 c) {
+            const uint32_t box = sb + (uint32_t)((q >> 2) * kBoxBytes) + (uint32_t)r * 128u;
+            const uint32_t c0 = (uint32_t)(2 * (q & 3));
+            st_shared_v4(box + ((c0 ^ sw) << 4), dequant8_e4m3(c.x, c.y, sc));
+            st_shared_v4(box + (((c0 + 1u) ^ sw) << 4), dequant8_e4m3(c.z, c.w, sc));
+          };
+#pragma unroll 1
+          for (int c = 0; c < 8; ++c) {  // columns 0..127 -> boxes 0, 1
+            const int q = (c + r) & 7;
+            put(q, ld_shared_v4(codes + (uint32_t)q * 16u));
           }
-          __syncwarp();
-          if (lane == 0) mbar_arrive(smem_addr(&misc->conv_sync));
-          if (!W.wait_warp(&misc->conv_sync, k & 1)) {
-            ok = false;
-            break;
+#pragma unroll 1
+          for (int c = 0; c < 4; ++c) {  // columns 128..191 -> box 2, over code box 0's row
+            const int q = 8 + ((c + r) & 3);
+            put(q, ld_shared_v4(codes + kF8CodeBoxBytes + (uint32_t)(q - 8) * 16u));
           }
+          uint4 last[4];  // columns 192..255: read all, then box 3 over code box 1's row
 #pragma unroll
+          for (int c = 0; c < 4; ++c)
+            last[c] = ld_shared_v4(codes + kF8CodeBoxBytes + 64u + (uint32_t)((c + r) & 3) * 16u);
 #pragma unroll
-          for (int u = 0; u < 16; ++u) {
-            const int id = 64 * u + ct, row = id >> 4, qc = id & 15;
-            const uint32_t soff = a.topk > 0 ? (uint32_t)((row >> 2) * 128 + (row & 3) * 16) : (uint32_t)(row * 16);
-            const float sc = __uint_as_float(ld_shared_u32(sb + kF8ScaleStageOff + soff));
-            // latent box qc / 4, columns 16 (qc % 4) .. + 15 of it: 16-byte chunks 2 (qc % 4) and + 1
-            const uint32_t box = sb + (uint32_t)((qc >> 2) * kBoxBytes + row * 128);
-            const uint32_t c0 = (uint32_t)(2 * (qc & 3)), sw = (uint32_t)(row & 7);
-            st_shared_v4(box + ((c0 ^ sw) << 4), dequant8_e4m3(cw[u].x, cw[u].y, sc));
-            st_shared_v4(box + (((c0 + 1u) ^ sw) << 4), dequant8_e4m3(cw[u].z, cw[u].w, sc));
-          }
+          for (int c = 0; c < 4; ++c) put(12 + ((c + r) & 3), last[c]);
           fence_proxy_async_smem();  // read by the tensor core
           __syncwarp();
           if (lane == 0) mbar_arrive(smem_addr(&misc->conv_full[s]));
