@@ -39,7 +39,7 @@ using namespace ptx;
 
 constexpr int kThreads = 128;
 constexpr int kBox = 128 * 128;            // bytes of one 128-row x 64-column bf16 box
-constexpr int kAbsorbSmem = 6 * kBox;      // Q (2 boxes) + one half of W_UK (4 boxes)
+constexpr int kAbsorbSmem = 6 * kBox;      // Q (2 boxes; q_pe after the MMAs) + one half of W_UK (4 boxes)
 constexpr int kUnStages = 3;
 constexpr int kUnStageBytes = 4 * kBox;    // O chunk (2 boxes) + W_UV chunk (2 boxes)
 constexpr int kUnSmem = kUnStages * kUnStageBytes;
@@ -50,6 +50,7 @@ constexpr uint32_t kErrTimeoutBit = 0x8u;
 struct Maps {
   CUtensorMap act;  // activations: [T rows, H * width columns] bf16
   CUtensorMap w;    // wkv_b: [H * 256 rows, 512 columns] bf16
+  CUtensorMap out;  // result: [T rows, H * out_width columns] bf16 (TMA stores; rows past T are not written)
 };
 
 struct Args {
@@ -97,6 +98,40 @@ MLA_DEV void store_row_bf16(__nv_bfloat16* dst, const uint32_t (&r)[32]) {
                       pack_bf16x2(__uint_as_float(r[8 * u + 2]), __uint_as_float(r[8 * u + 3])),
                       pack_bf16x2(__uint_as_float(r[8 * u + 4]), __uint_as_float(r[8 * u + 5])),
                       pack_bf16x2(__uint_as_float(r[8 * u + 6]), __uint_as_float(r[8 * u + 7])));
+}
+
+// TMA store of a 2-D box from shared memory (completion tracked by the
+// issuing thread's bulk async-group).
+MLA_DEV void tma_store_2d(const CUtensorMap* map, uint32_t src, int32_t c0, int32_t c1) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group [%0, {%1, %2}], [%3];" ::"l"(map), "r"(c0),
+               "r"(c1), "r"(src)
+               : "memory");
+}
+MLA_DEV void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+MLA_DEV void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+
+// The epilogue's staging: this thread's TMEM lane (token row `row`) holds
+// 32 * nchunks fp32 columns; they are rounded to bf16 and written as row
+// `row` of 64-column boxes (128 bytes per row, 128-byte swizzle) at `boxes`,
+// the layout a TMA store of those boxes reads.
+MLA_DEV void stage_rows_bf16(uint32_t taddr, int nchunks, uint32_t boxes, int row) {
+#pragma unroll 1
+  for (int c = 0; c < nchunks; ++c) {
+    uint32_t r[32];
+    tmem_ld_32x32b_32(taddr + 32u * c, r);
+    tmem_wait_ld();
+    const uint32_t rowp = boxes + (uint32_t)((c >> 1) * kBox + row * 128);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const uint32_t j = (uint32_t)((c & 1) * 4 + u);  // 16-byte chunk of the 128-byte row
+      st_shared_v4(rowp + ((j ^ (uint32_t)(row & 7)) << 4),
+                   make_uint4(pack_bf16x2(__uint_as_float(r[8 * u + 0]), __uint_as_float(r[8 * u + 1])),
+                              pack_bf16x2(__uint_as_float(r[8 * u + 2]), __uint_as_float(r[8 * u + 3])),
+                              pack_bf16x2(__uint_as_float(r[8 * u + 4]), __uint_as_float(r[8 * u + 5])),
+                              pack_bf16x2(__uint_as_float(r[8 * u + 6]), __uint_as_float(r[8 * u + 7]))));
+    }
+  }
+  fence_proxy_async_smem();  // read by the TMA store
 }
 
 MLA_DEV uint32_t aligned_base(uint8_t* raw) { return (smem_addr(raw) + (kAlignPad - 1)) & ~(uint32_t)(kAlignPad - 1); }
@@ -164,6 +199,11 @@ __global__ void __launch_bounds__(kThreads, 1) mla_absorb_q_kernel(const __grid_
                smem_desc_sw128(sb + ks * 2048, kBox, 1024), idesc, ks > 0 ? 1u : 0u);
       mma_commit(done);
       ok = wait_bounded(done, 0);
+      // q_pe passes through: into the Q buffer, which the MMAs are done with
+      if (ok && nh == 0) {
+        mbar_arrive_expect_tx(smem_addr(&bars.full[1]), kBox);
+        tma_load_2d(sa, &maps.act, h * 192 + 128, m0, smem_addr(&bars.full[1]));
+      }
     } else {
       wait_bounded(full, 0);  // give the copies in flight a last chance to land
     }
@@ -171,23 +211,20 @@ __global__ void __launch_bounds__(kThreads, 1) mla_absorb_q_kernel(const __grid_
   }
   __syncthreads();
   tc_fence_after();
-  if (!bars.fail) {
-    const int t = m0 + 32 * warp + lane;
-    const bool valid = t < a.tokens;
-    const size_t row = (size_t)t * a.heads + h;
-#pragma unroll 1
-    for (int c = 0; c < 8; ++c) {
-      uint32_t r[32];
-      tmem_ld_32x32b_32(tmem + ((uint32_t)(32 * warp) << 16) + 32u * c, r);
-      tmem_wait_ld();
-      if (valid) store_row_bf16(a.out + row * (kDLatent + kDRope) + nh * 256 + 32 * c, r);
-    }
-    if (valid && nh == 0) {  // the rope part of the query passes through unchanged
-      const uint4* src = reinterpret_cast<const uint4*>(a.q + row * 192 + 128);
-      uint4* dst = reinterpret_cast<uint4*>(a.out + row * (kDLatent + kDRope) + kDLatent);
+  // epilogue: the 256 result columns, rounded to bf16, staged over the W_UK
+  // boxes (the MMAs are done with them) and written by four TMA stores
+  if (!bars.fail) stage_rows_bf16(tmem + ((uint32_t)(32 * warp) << 16), 8, sb, 32 * warp + lane);
+  __syncthreads();
+  if (threadIdx.x == 0 && !bars.fail) {
+    const int col = h * (kDLatent + kDRope) + nh * 256;
 #pragma unroll
-      for (int u = 0; u < 8; ++u) dst[u] = src[u];
+    for (int b = 0; b < 4; ++b) tma_store_2d(&maps.out, sb + b * kBox, col + 64 * b, m0);
+    if (nh == 0) {
+      if (wait_bounded(smem_addr(&bars.full[1]), 0)) tma_store_2d(&maps.out, sa, h * (kDLatent + kDRope) + kDLatent, m0);
+      else record_timeout(&bars, a.error);
     }
+    bulk_commit();
+    bulk_wait_read();  // the stores have read shared memory before the CTA can exit
   }
   teardown(&bars, tmem, 256);
 }
@@ -251,17 +288,15 @@ __global__ void __launch_bounds__(kThreads, 1) mla_unabsorb_o_kernel(const __gri
   }
   __syncthreads();
   tc_fence_after();
-  if (!bars.fail) {
-    const int t = m0 + 32 * warp + lane;
-    const bool valid = t < a.tokens;
-    const size_t row = (size_t)t * a.heads + h;
-#pragma unroll 1
-    for (int c = 0; c < 4; ++c) {
-      uint32_t r[32];
-      tmem_ld_32x32b_32(tmem + ((uint32_t)(32 * warp) << 16) + 32u * c, r);
-      tmem_wait_ld();
-      if (valid) store_row_bf16(a.out + row * 128 + 32 * c, r);
-    }
+  // epilogue: 128 result columns in two boxes staged over stage 0 (the MMAs
+  // are done with it), written by two TMA stores
+  if (!bars.fail) stage_rows_bf16(tmem + ((uint32_t)(32 * warp) << 16), 4, base, 32 * warp + lane);
+  __syncthreads();
+  if (threadIdx.x == 0 && !bars.fail) {
+#pragma unroll
+    for (int b = 0; b < 2; ++b) tma_store_2d(&maps.out, base + b * kBox, h * 128 + 64 * b, m0);
+    bulk_commit();
+    bulk_wait_read();
   }
   teardown(&bars, tmem, 128);
 }
@@ -278,8 +313,10 @@ mla_status_t check(const mla_absorb_desc_t* d) {
   return MLA_OK;
 }
 
-// act: [T rows, H * width columns]; w: wkv_b as [H * 256 rows, 512 columns].
-bool encode_maps(Maps* m, const void* act, int tokens, int heads, int width, const void* wkv_b) {
+// act: [T rows, H * width columns]; w: wkv_b as [H * 256 rows, 512 columns];
+// out: [T rows, H * out_width columns].
+bool encode_maps(Maps* m, const void* act, int tokens, int heads, int width, const void* wkv_b, void* out,
+                 int out_width) {
   PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
   if (!enc) return false;
   cuuint32_t box[2] = {64, 128};
@@ -288,11 +325,16 @@ bool encode_maps(Maps* m, const void* act, int tokens, int heads, int width, con
   cuuint64_t astr[1] = {(cuuint64_t)heads * width * 2};
   cuuint64_t wdims[2] = {(cuuint64_t)kDLatent, (cuuint64_t)heads * 256};
   cuuint64_t wstr[1] = {(cuuint64_t)kDLatent * 2};
+  cuuint64_t odims[2] = {(cuuint64_t)heads * out_width, (cuuint64_t)tokens};
+  cuuint64_t ostr[1] = {(cuuint64_t)heads * out_width * 2};
   return enc(&m->act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(act), adims, astr, box, elem,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS &&
          enc(&m->w, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(wkv_b), wdims, wstr, box, elem,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS &&
+         enc(&m->out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, out, odims, ostr, box, elem, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -315,7 +357,8 @@ extern "C" MLA_API mla_status_t mla_absorb_query(const mla_absorb_desc_t* desc, 
       !gemm::aligned(error_word, 4))
     return MLA_ERR_INVALID_ARG;
   gemm::Maps maps;
-  if (!gemm::encode_maps(&maps, q, desc->num_tokens, desc->num_heads, 192, wkv_b)) return MLA_ERR_CUDA;
+  if (!gemm::encode_maps(&maps, q, desc->num_tokens, desc->num_heads, 192, wkv_b, q_abs, kDLatent + kDRope))
+    return MLA_ERR_CUDA;
   const int smem = gemm::kAbsorbSmem + gemm::kAlignPad;
   if (gemm::set_smem((const void*)gemm::mla_absorb_q_kernel, smem) != cudaSuccess) return MLA_ERR_CUDA;
   gemm::Args a{static_cast<const __nv_bfloat16*>(q), static_cast<__nv_bfloat16*>(q_abs), error_word,
@@ -336,7 +379,8 @@ extern "C" MLA_API mla_status_t mla_unabsorb_output(const mla_absorb_desc_t* des
       !gemm::aligned(error_word, 4))
     return MLA_ERR_INVALID_ARG;
   gemm::Maps maps;
-  if (!gemm::encode_maps(&maps, o_lat, desc->num_tokens, desc->num_heads, kDLatent, wkv_b)) return MLA_ERR_CUDA;
+  if (!gemm::encode_maps(&maps, o_lat, desc->num_tokens, desc->num_heads, kDLatent, wkv_b, out, 128))
+    return MLA_ERR_CUDA;
   const int smem = gemm::kUnSmem + gemm::kAlignPad;
   if (gemm::set_smem((const void*)gemm::mla_unabsorb_o_kernel, smem) != cudaSuccess) return MLA_ERR_CUDA;
   gemm::Args a{nullptr, static_cast<__nv_bfloat16*>(out), error_word, desc->num_tokens, desc->num_heads};
