@@ -20,16 +20,55 @@ constexpr int kRowsPerTask = 128;  // heads handled by one worker (one TMEM lane
 constexpr int kMaxHeads = 128;
 
 // Plan buffer (int32 words):
-//   [0] device error word   [1] number of tasks T   [2] pages per worker (quota)
-//   [3] total pages         [4] workers             [5] heads     [6..7] reserved
-//   [8 .. 8+T]      prefix[t]: first global page of task t (prefix[T] = total)
-//   [9+T .. 9+2T)   ntok[t]: tokens (or index slots) of task t after validation
+//   [0] device error word   [1] number of tasks T   [2] quota of group 0
+//   [3] total pages         [4] workers             [5] heads
+//   [6] worker groups G     [7] workers per group Wg
+//   [8 .. 8+T]      prefix[u]: first global page of plan position u (prefix[T] = total)
+//   [9+T .. 9+2T)   ntok[u]: tokens (or index slots) of position u after validation
 constexpr int kPlanHeader = 8;
 constexpr int kPlanErr = 0, kPlanTasks = 1, kPlanQuota = 2, kPlanTotal = 3, kPlanWorkers = 4, kPlanHeads = 5;
+constexpr int kPlanGroups = 6, kPlanGroupWorkers = 7;
 
 __host__ __device__ inline int plan_prefix_off() { return kPlanHeader; }
 __host__ __device__ inline int plan_ntok_off(int tasks) { return kPlanHeader + tasks + 1; }
 __host__ __device__ inline int plan_words(int tasks) { return kPlanHeader + 2 * tasks + 1; }
+
+// Worker groups: with several dense query tokens per sequence (2..8, no
+// top-k) and at least 4 workers per token, the workers form G = Sq equal
+// groups and group g takes token g of every sequence. The tokens of one
+// sequence read the same pages, and the groups walk them in step, so a page
+// fetched for one token is still in L2 for the others. Otherwise G = 1.
+__host__ __device__ inline int plan_groups(int q_len, int topk, int workers) {
+  return (q_len >= 2 && q_len <= 8 && topk == 0 && workers / q_len >= 4) ? q_len : 1;
+}
+
+// Plan order: with G > 1 groups, position u holds query token u / B of
+// sequence u % B (token-major, so a group's positions are contiguous); with
+// G = 1 it is query row u = b * Sq + i.
+struct TaskMap {
+  int groups, batch, q_len;
+  __host__ __device__ int seq(int u) const { return groups > 1 ? u % batch : u / q_len; }
+  __host__ __device__ int tok(int u) const { return groups > 1 ? u / batch : u % q_len; }
+  __host__ __device__ int row(int u) const { return groups > 1 ? (u % batch) * q_len + u / batch : u; }
+};
+
+// Group g of a plan: positions [t0, t1), global pages [base, end), split
+// over workers [w0, w0 + Wg) in runs of `quota` pages.
+struct PlanGroup {
+  int t0, t1, base, end, quota, w0;
+};
+__device__ inline PlanGroup plan_group(const int32_t* plan, int g) {
+  const int T = plan[kPlanTasks], G = plan[kPlanGroups], Wg = plan[kPlanGroupWorkers];
+  const int32_t* prefix = plan + plan_prefix_off();
+  PlanGroup r;
+  r.t0 = g * (T / G);
+  r.t1 = r.t0 + T / G;
+  r.base = prefix[r.t0];
+  r.end = prefix[r.t1];
+  r.quota = max(1, (r.end - r.base + Wg - 1) / Wg);
+  r.w0 = g * Wg;
+  return r;
+}
 
 constexpr uint32_t kErrSeqLen = 0x1u, kErrPageId = 0x2u, kErrIndex = 0x4u, kErrTimeout = 0x8u;
 

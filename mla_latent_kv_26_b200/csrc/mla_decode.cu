@@ -172,23 +172,29 @@ struct Waiter {
   }
 };
 
-// The worker's contiguous range of global pages, walked task by task.
+// The worker's contiguous range of global pages (inside its group's
+// positions), walked task by task in plan order.
 struct Cursor {
   const int32_t* prefix;
-  int T, lo, hi, t;
+  int T, lo, hi, t, tend;
 
   MLA_DEV void init(const int32_t* plan, int worker) {
     T = plan[kPlanTasks];
-    const int quota = plan[kPlanQuota];
-    const int total = plan[kPlanTotal];
     prefix = plan + plan_prefix_off();
-    lo = worker * quota;
-    hi = min(lo + quota, total);
-    if (lo >= total || T <= 0) {
-      t = T;
+    const int G = plan[kPlanGroups], Wg = plan[kPlanGroupWorkers];
+    const int g = worker / Wg;
+    t = tend = T;
+    lo = hi = 0;
+    if (T <= 0 || g >= G) return;  // no tasks, or one of the workers left over by the grouping
+    const PlanGroup grp = plan_group(plan, g);
+    lo = grp.base + (worker - grp.w0) * grp.quota;
+    hi = min(lo + grp.quota, grp.end);
+    tend = grp.t1;
+    if (lo >= grp.end) {
+      t = tend;
       return;
     }
-    int a = 0, b = T - 1;  // largest t with prefix[t] <= lo
+    int a = grp.t0, b = grp.t1 - 1;  // largest t in the group with prefix[t] <= lo
     while (a < b) {
       const int mid = (a + b + 1) >> 1;
       if (prefix[mid] <= lo) a = mid;
@@ -197,7 +203,7 @@ struct Cursor {
     t = a;
   }
   MLA_DEV bool next(int& task, int& pg0, int& pg1, bool& split) {
-    while (t < T && prefix[t] < hi) {
+    while (t < tend && prefix[t] < hi) {
       const int cur = t++;
       const int p0 = prefix[cur], p1 = prefix[cur + 1];
       const int a = max(lo, p0), b = min(hi, p1);
@@ -287,6 +293,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kF8 ? kThreadsF8 : k
   Cursor cur;
   cur.init(a.plan, worker);
   const int T = cur.T;
+  const TaskMap tmap{a.plan[kPlanGroups], a.batch, a.q_len};
   const int32_t* ntok_arr = a.plan + plan_ntok_off(T);
   int task = 0, pg0 = 0, pg1 = 0;
   bool split = false;
@@ -308,7 +315,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kF8 ? kThreadsF8 : k
   // shared memory.
   auto write_q = [&](int half) {
     const int row = quad * 32 + lane;
-    const size_t qrow = (size_t)task * a.heads + row;
+    const size_t qrow = (size_t)tmap.row(task) * a.heads + row;
     const bool valid = row < a.heads;
     const uint4* src = reinterpret_cast<const uint4*>(a.q + qrow * kDQK + vcol0 + half * 128);
     uint32_t qv[64];
@@ -361,7 +368,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kF8 ? kThreadsF8 : k
   // Epilogue for a 16-lane half: out / partials of rows `row` (per thread), columns th*128 + [0,128).
   auto write_rows = [&](uint32_t lanes, int row, float inv, float lse, bool write_lse) {
     const bool valid = row < a.heads;
-    const size_t qrow = (size_t)task * a.heads + row;
+    const size_t qrow = (size_t)tmap.row(task) * a.heads + row;
 #pragma unroll 1
     for (int c = 0; c < 4; ++c) {
       uint32_t o[32];
@@ -408,7 +415,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kF8 ? kThreadsF8 : k
     // ------------------------------------------------------------ producer
     int k = 0;
     while (cur.next(task, pg0, pg1, split)) {
-      const int b = task / a.q_len, qi = task % a.q_len;
+      const int b = tmap.seq(task), qi = tmap.tok(task);
       const int ntok = ntok_arr[task];
       const int32_t* bt_row = a.block_table + (size_t)b * a.max_pages_per_seq;
       if (a.topk == 0) {

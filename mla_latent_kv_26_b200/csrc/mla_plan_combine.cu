@@ -5,9 +5,10 @@
 
 namespace mla {
 
-// One block of 1024 threads. Task t = b * Sq + i gets ntok[t] tokens (index
-// slots when sparse) and ceil(ntok/64) pages; prefix[] lays the tasks' pages
-// end to end; worker w owns global pages [w*quota, (w+1)*quota).
+// One block of 1024 threads. Plan position u (query token TaskMap::tok(u)
+// of sequence TaskMap::seq(u)) gets ntok[u] tokens (index slots when sparse)
+// and ceil(ntok/64) pages; prefix[] lays the positions' pages end to end;
+// worker j of group g owns the group's pages [j*quota_g, (j+1)*quota_g).
 __global__ void __launch_bounds__(1024) mla_plan_kernel(PlanArgs a) {
   __shared__ int s_scan[1024];
   __shared__ int s_carry;
@@ -22,11 +23,13 @@ __global__ void __launch_bounds__(1024) mla_plan_kernel(PlanArgs a) {
   }
   __syncthreads();
   const long long cap = (long long)a.max_pages_per_seq * kPage;
+  const int G = plan_groups(a.q_len, a.topk, a.workers);
+  const TaskMap map{G, a.batch, a.q_len};
   for (int base = 0; base < T; base += 1024) {
     const int t = base + tid;
     int pages = 0;
     if (t < T) {
-      const int b = t / a.q_len, i = t % a.q_len;
+      const int b = map.seq(t), i = map.tok(t);
       const int L = a.seq_lens[b];
       const bool ok = L >= 0 && (long long)L <= cap;
       int n = 0;
@@ -51,15 +54,16 @@ __global__ void __launch_bounds__(1024) mla_plan_kernel(PlanArgs a) {
   if (tid == 0) {
     const int total = s_carry;
     prefix[T] = total;
-    const int quota = max(1, (total + a.workers - 1) / a.workers);
+    const int Wg = a.workers / G;
+    const int pages0 = prefix[T / G];  // pages of group 0 (prefix[0] = 0)
     a.plan[kPlanErr] = (int32_t)s_err;
     a.plan[kPlanTasks] = T;
-    a.plan[kPlanQuota] = quota;
+    a.plan[kPlanQuota] = max(1, (pages0 + Wg - 1) / Wg);
     a.plan[kPlanTotal] = total;
     a.plan[kPlanWorkers] = a.workers;
     a.plan[kPlanHeads] = a.heads;
-    a.plan[6] = 0;
-    a.plan[7] = 0;
+    a.plan[kPlanGroups] = G;
+    a.plan[kPlanGroupWorkers] = Wg;
   }
 }
 
@@ -71,17 +75,19 @@ __global__ void __launch_bounds__(1024) mla_plan_kernel(PlanArgs a) {
 // lse = M + ln sum_w exp(lse_w - M), out = sum_w exp(lse_w - lse) * o_w.
 __global__ void __launch_bounds__(256) mla_combine_kernel(CombineArgs a) {
   const int T = a.plan[kPlanTasks];
-  const int quota = a.plan[kPlanQuota];
   const int t = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int h = blockIdx.y * 8 + warp;
   if (t >= T || h >= a.heads) return;
+  const int G = a.plan[kPlanGroups];
+  const PlanGroup grp = plan_group(a.plan, t / (T / G));
   const int32_t* prefix = a.plan + plan_prefix_off();
   const int p0 = prefix[t], p1 = prefix[t + 1];
-  const size_t row = (size_t)t * a.heads + h;
+  const TaskMap map{G, T / G, G};  // with G > 1, q_len = G; with G = 1, row(t) = t
+  const size_t row = (size_t)map.row(t) * a.heads + h;
   __nv_bfloat16* orow = a.out + row * kDLatent;
-  const int w0 = p0 / quota;
-  const int w1 = p1 > p0 ? (p1 - 1) / quota : w0;
+  const int w0 = grp.w0 + (p0 - grp.base) / grp.quota;
+  const int w1 = p1 > p0 ? grp.w0 + (p1 - 1 - grp.base) / grp.quota : w0;
   if (p1 > p0 && w0 == w1) return;
 
   float m[2] = {-INFINITY, -INFINITY};

@@ -317,34 +317,58 @@ def test_lse_merge_two_scalars_by_hand():
     ([131072] * 4, 1, False, 2048, 74),
     ([3, 5], 2, True, 0, 1),
     ([], 1, False, 0, 3),
+    ([4096, 65536, 1, 65, 129, 700], 2, True, 0, 74),   # grouped: 2 x 37 workers
+    ([5000, 64, 3, 9000], 3, True, 0, 74),              # grouped: 3 x 24, 2 idle
+    ([5000, 64, 3, 9000], 2, False, 0, 74),             # grouped, not causal
+    ([5000, 64], 9, True, 0, 74),                       # q_len 9: not grouped
+    ([300, 3000], 2, True, 2048, 74),                   # sparse: not grouped
 ])
 def test_plan_covers_every_page_once_within_quota(lens, Sq, causal, topk, P):
     maxp = max([(L + 63) // 64 for L in lens] + [1])
     plan = split_plan(lens, q_len=Sq, causal=causal, topk=topk, max_pages_per_seq=maxp, num_pairs=P)
+    G, Wg = plan["groups"], plan["workers_per_group"]
+    grouped = 2 <= Sq <= 8 and topk == 0 and P // Sq >= 4
+    assert G == (Sq if grouped else 1) and Wg == P // G
+    T = len(lens) * Sq
+    # plan order: a permutation of the query rows; token-major when grouped
+    assert sorted(plan["task_rows"]) == list(range(T))
+    for u, r in enumerate(plan["task_rows"]):
+        assert r == ((u % len(lens)) * Sq + u // len(lens) if grouped else u)
     covered = {}
     slots = set()
     for p, items in enumerate(plan["items"]):
         load = 0
+        g = p // Wg if Wg else 0
         for (t, a, b, slot) in items:
             assert 0 <= a < b <= plan["task_pages"][t]
+            assert g < G and g * (T // G) <= t < (g + 1) * (T // G)   # a worker stays in its group
             for pg in range(a, b):
                 assert (t, pg) not in covered
                 covered[(t, pg)] = p
             load += b - a
             assert slot == p + t and slot not in slots
             slots.add(slot)
-        assert load <= plan["quota"]
+        if items:
+            assert load <= plan["quotas"][g]
     want = {(t, pg) for t, n in enumerate(plan["task_pages"]) for pg in range(n)}
     assert set(covered) == want
     assert plan["total_pages"] == len(want)
     # tokens per task from the definition, by brute force
     for t, n in enumerate(plan["task_tokens"]):
-        b, i = divmod(t, Sq)
+        b, i = divmod(plan["task_rows"][t], Sq)
         L = lens[b]
         exp = topk if topk else (max(L - Sq + i + 1, 0) if causal else L)
         assert n == exp
         assert plan["task_pages"][t] == -(-n // 64)
         assert plan["splits"][t] == len({covered[(t, pg)] for pg in range(plan["task_pages"][t])})
+    if grouped and not causal:
+        # every token of a sequence reads the same pages: worker j of every
+        # group gets the same (sequence, page range) items
+        B = len(lens)
+        for j in range(Wg):
+            seen = [[(plan["task_rows"][t] // Sq, a, b) for (t, a, b, _) in plan["items"][g * Wg + j]]
+                    for g in range(G)]
+            assert all(s == seen[0] for s in seen)
 
 
 def test_plan_flags_out_of_range_lengths():

@@ -99,6 +99,22 @@ def test_causal_pair(dev, heads, lens):
     check_case(d, dev, 2, f"causal H{heads} {lens} one worker")
 
 
+@pytest.mark.parametrize("q_len,causal,lens", [(3, True, [65, 129, 1, 2, 700]), (4, False, [64, 193, 5]),
+                                                (2, True, [1, 65, 4097, 3000])])
+@pytest.mark.parametrize("num_sms", [0, 16, 14])
+def test_query_token_groups(dev, q_len, causal, lens, num_sms):
+    """Several query tokens per sequence: with enough workers the plan puts
+    token g of every sequence in worker group g (16 SMs = 8 workers is the
+    threshold for two tokens, 14 SMs stays ungrouped); lengths 64 k + 1 give
+    the tokens different page counts under the causal mask."""
+    from mla_latent_kv_26_b200.workloads import small
+
+    d = small(batch=len(lens), heads=128, q_len=q_len, causal=causal, lens=lens, seed=40 + q_len)
+    _, _, dec = check_case(d, dev, num_sms, f"Sq={q_len} causal={causal} sms{num_sms}")
+    plan = dec.plan.view(torch.int32).cpu()
+    assert plan[6].item() == oracle.plan.plan_groups(q_len=q_len, topk=0, num_pairs=dec.num_workers)
+
+
 def test_non_causal_pair(dev):
     from mla_latent_kv_26_b200.workloads import small
 
@@ -175,7 +191,8 @@ def test_plan_matches_oracle_schedule(dev):
     from mla_latent_kv_26_b200.workloads import small
 
     for lens, Sq, causal, topk, sms in [([1024, 32768, 5000, 77, 0, 64], 1, False, 0, 10), ([4096, 600], 2, True, 0, 0),
-                                         ([9000, 9000], 1, False, 2048, 6)]:
+                                         ([9000, 9000], 1, False, 2048, 6), ([65, 129, 1, 700], 3, True, 0, 0),
+                                         ([4096, 600], 2, True, 0, 14)]:
         d = small(batch=len(lens), heads=128, q_len=Sq, causal=causal, lens=lens, topk=topk, seed=3)
         out, lse, st, bits, dec = run_gpu(d, dev, sms)
         plan = dec.plan.view(torch.int32).cpu()
@@ -186,6 +203,7 @@ def test_plan_matches_oracle_schedule(dev):
         assert plan[2].item() == ref["quota"]
         assert plan[3].item() == ref["total_pages"]
         assert plan[4].item() == dec.num_workers
+        assert plan[6].item() == ref["groups"] and plan[7].item() == ref["workers_per_group"]
         assert plan[8:8 + T + 1].tolist() == ref["prefix"]
         assert plan[9 + T:9 + 2 * T].tolist() == ref["task_tokens"]
 
