@@ -83,6 +83,7 @@ struct DecodeArgs {
   const int32_t* block_table;   // [B, max_pages_per_seq]
   const int32_t* seq_lens;      // [B]
   const int32_t* indices;       // [B, Sq, topk] or nullptr
+  const uint8_t* cache;         // the cache's first byte (row copies of gathered tokens)
   __nv_bfloat16* out;           // [B, Sq, H, 512]
   float* lse;                   // [B, Sq, H]
   float* part_o;                // [slots, H, 512]

@@ -241,6 +241,7 @@ mla_status_t decode_impl(const mla_decode_desc_t* desc, void* plan, const void* 
   a.block_table = block_table;
   a.seq_lens = seq_lens;
   a.indices = topk_indices;
+  a.cache = static_cast<const uint8_t*>(kv_cache);
   a.out = reinterpret_cast<__nv_bfloat16*>(out);
   a.lse = lse;
   a.part_o = reinterpret_cast<float*>(workspace);

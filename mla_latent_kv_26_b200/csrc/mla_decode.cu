@@ -194,11 +194,24 @@ struct Cursor {
       t = tend;
       return;
     }
-    int a = grp.t0, b = grp.t1 - 1;  // largest t in the group with prefix[t] <= lo
+    // largest t in the group with prefix[t] <= lo: a 32-way search by the
+    // whole warp (one round of loads per factor 32 of the range instead of
+    // one per halving; every lane of the calling warp takes part)
+    const int lane = threadIdx.x & 31;
+    int a = grp.t0, b = grp.t1 - 1;
     while (a < b) {
-      const int mid = (a + b + 1) >> 1;
-      if (prefix[mid] <= lo) a = mid;
-      else b = mid - 1;
+      const int step = (b - a + 31) / 32;
+      const int q = min(a + (lane + 1) * step, b);
+      const unsigned le = __ballot_sync(~0u, prefix[q] <= lo);  // a prefix of the lanes (prefix is nondecreasing)
+      const int m = __popc(le);
+      const int qm = __shfl_sync(~0u, q, max(m - 1, 0));  // last probe at or before the answer
+      const int qn = __shfl_sync(~0u, q, min(m, 31));     // first probe after it (m < 32)
+      if (m == 0) {
+        b = qn - 1;
+      } else {
+        a = qm;                      // m == 32: the last probe is b itself, so a = b
+        if (m < 32) b = qn - 1;
+      }
     }
     t = a;
   }
@@ -245,7 +258,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kF8 ? kThreadsF8 : k
   }
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(smem_addr(&misc->full[s]), 1);
+      // bf16 gathers: 32 cp.async arrivals + lane 0's arrive with the TMA bytes
+      mbar_init(smem_addr(&misc->full[s]), (!kF8 && a.topk > 0) ? 33 : 1);
       mbar_init(smem_addr(&misc->empty[s]), 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -463,63 +477,119 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kF8 ? kThreadsF8 : k
       } else {
         const int32_t* idx_row = a.indices + (size_t)(b * a.q_len + qi) * a.topk;
         const int L = a.seq_lens[b];
-        for (int tile = pg0; tile < pg1; ++tile, ++k) {
-          int rows[2];
-          bool valid[2];
+        // Index slots in batches of 4 tiles (8 per lane): the next batch's
+        // indices are loaded before this batch's block-table lookups, and the
+        // 8 lookups of a batch go out together, so a batch costs about one
+        // round trip to memory instead of two per tile.
+        int nidx[8];
+        auto load_idx = [&](int t0, int (&dst)[8]) {
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const int slot = tile * kPage + lane + 32 * h;
-            const int idx = slot < ntok ? idx_row[slot] : -1;
-            const bool in_range = idx >= 0 && idx < L;
-            if (slot < ntok && !in_range && idx != -1) atomicOr(W.err, kErrIndex);
-            int pid = 0;
-            bool pok = false;
-            if (in_range) {
-              pid = bt_row[idx / kPage];
-              pok = (unsigned)pid < (unsigned)a.num_pages;
-              if (!pok) atomicOr(W.err, kErrPageId);
+          for (int h = 0; h < 8; ++h) {
+            const int slot = t0 * kPage + 32 * h + lane;
+            dst[h] = (t0 + (h >> 1) < pg1 && slot < ntok) ? idx_row[slot] : -1;
+          }
+        };
+        load_idx(pg0, nidx);
+        for (int t0 = pg0; t0 < pg1; t0 += 4) {
+          int idx[8];
+#pragma unroll
+          for (int h = 0; h < 8; ++h) idx[h] = nidx[h];
+          if (t0 + 4 < pg1) load_idx(t0 + 4, nidx);
+          int rows8[8];
+          bool valid8[8];
+#pragma unroll
+          for (int h = 0; h < 8; ++h) {
+            const int slot = t0 * kPage + 32 * h + lane;
+            const bool in_range = idx[h] >= 0 && idx[h] < L;
+            if (t0 + (h >> 1) < pg1 && slot < ntok && !in_range && idx[h] != -1) atomicOr(W.err, kErrIndex);
+            const int pid = in_range ? bt_row[idx[h] / kPage] : 0;
+            const bool pok = in_range && (unsigned)pid < (unsigned)a.num_pages;
+            if (in_range && !pok) atomicOr(W.err, kErrPageId);
+            rows8[h] = pok ? pid * kPage + (idx[h] % kPage) : 0;
+            valid8[h] = pok;
+          }
+#pragma unroll
+          for (int tt = 0; tt < 4; ++tt) {
+            if (t0 + tt >= pg1) break;
+            const int rows[2] = {rows8[2 * tt], rows8[2 * tt + 1]};
+            const uint64_t mask = (uint64_t)__ballot_sync(~0u, valid8[2 * tt]) |
+                                  ((uint64_t)__ballot_sync(~0u, valid8[2 * tt + 1]) << 32);
+            int r[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const int src = (4 * lane + u) & 31;
+              const int r0 = __shfl_sync(~0u, rows[0], src);
+              const int r1 = __shfl_sync(~0u, rows[1], src);
+              r[u] = lane < 8 ? r0 : r1;
             }
-            rows[h] = pok ? pid * kPage + (idx % kPage) : 0;
-            valid[h] = pok;
-          }
-          const uint64_t mask =
-              (uint64_t)__ballot_sync(~0u, valid[0]) | ((uint64_t)__ballot_sync(~0u, valid[1]) << 32);
-          int r[4];
+            const int s = k % kStages;
+            if (!W.wait_warp(&misc->empty[s], ((k / kStages) & 1) ^ 1)) goto producer_done;
+            const uint32_t fb = smem_addr(&misc->full[s]);
+            if constexpr (!kF8) {
+              // Two engines at once: tile::gather4 (TMA) brings latent boxes 0
+              // and 1 and the rope box, 16-byte cp.async copies by the whole
+              // warp bring latent boxes 2 and 3 (row t of the tile is rows[h]
+              // of lane t % 32, h = t / 32; lane l copies chunk l % 8 of box
+              // 2 + (l / 8) % 2 of row 2 i + l / 16, 128-byte swizzle: chunk ^
+              // (t % 8)), the layout a TMA load of those boxes writes. Per
+              // SM, each path alone moves a gathered tile at about the same
+              // rate, one warp issuing. The barrier expects 32 cp.async
+              // arrivals and lane 0's arrive with the TMA bytes.
+              const uint32_t dst = stage_base + s * kSB;
+              if (lane == 0) {
+                misc->stage_mask[s] = mask;
+                mbar_arrive_expect_tx(fb, 2 * kBoxBytes + kRopeBoxBytes);
+              }
+              __syncwarp();
+              if (lane < 16) {
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const int src = (4 * lane + u) & 31;
-            const int r0 = __shfl_sync(~0u, rows[0], src);
-            const int r1 = __shfl_sync(~0u, rows[1], src);
-            r[u] = lane < 8 ? r0 : r1;
-          }
-          const int s = k % kStages;
-          if (!W.wait_warp(&misc->empty[s], ((k / kStages) & 1) ^ 1)) goto producer_done;
-          const uint32_t fb = smem_addr(&misc->full[s]);
-          if (lane == 0) {
-            misc->stage_mask[s] = mask;
-            mbar_arrive_expect_tx(fb, kF8 ? kF8LoadBytes : kStageBytes);
-          }
-          __syncwarp();
-          if (lane < 16) {
-            // lane l gathers tile rows 4l .. 4l+3
-            const uint32_t dst = stage_base + s * kSB;
-            if constexpr (kF8) {
-              tma_gather4(dst + kF8CodeOff + lane * 4 * 128, &maps.row, vcol0, r[0], r[1], r[2], r[3], fb);
-              tma_gather4(dst + kF8CodeOff + kF8CodeBoxBytes + lane * 4 * 128, &maps.row, vcol0 + 128, r[0], r[1],
-                          r[2], r[3], fb);
-              tma_gather4(dst + kRopeOff + lane * 4 * 64, &maps.rope_row, kF8RopeOff + 64 * (int)crank, r[0], r[1],
-                          r[2], r[3], fb);
-              tma_gather4(dst + kF8ScaleStageOff + lane * 128, &maps.scale_row, kF8ScaleOff, r[0], r[1], r[2], r[3],
-                          fb);
-            } else {
-#pragma unroll
-              for (int bx = 0; bx < kVBoxes; ++bx)
-                tma_gather4(dst + bx * kBoxBytes + lane * 4 * 128, &maps.row, vcol0 + 64 * bx, r[0], r[1], r[2], r[3],
+                for (int bx = 0; bx < 2; ++bx)
+                  tma_gather4(dst + bx * kBoxBytes + lane * 4 * 128, &maps.row, vcol0 + 64 * bx, r[0], r[1], r[2], r[3],
+                              fb);
+                tma_gather4(dst + kRopeOff + lane * 4 * 64, &maps.rope_row, rcol0, r[0], r[1], r[2], r[3], fb);
+              }
+              const uint32_t bx = 2u + (uint32_t)((lane >> 3) & 1);
+              const uint32_t cc = (uint32_t)(lane & 7);
+              const size_t col_off = (size_t)(vcol0 + 64 * (int)bx + 8 * (int)cc) * 2;
+#pragma unroll 4
+              for (int i2 = 0; i2 < kPage / 2; ++i2) {
+                const int t = 2 * i2 + (lane >> 4);
+                const int rid = __shfl_sync(~0u, t < 32 ? rows[0] : rows[1], t & 31);
+                cp_async_16(dst + bx * kBoxBytes + (uint32_t)t * 128u + ((cc ^ (uint32_t)(t & 7)) << 4),
+                            a.cache + (size_t)rid * (kDQK * 2) + col_off);
+              }
+              cp_async_arrive_noinc(fb);
+              __syncwarp();
+              ++k;
+              continue;
+            }
+            if (lane == 0) {
+              misc->stage_mask[s] = mask;
+              mbar_arrive_expect_tx(fb, kF8 ? kF8LoadBytes : kStageBytes);
+            }
+            __syncwarp();
+            if (lane < 16) {
+              // lane l gathers tile rows 4l .. 4l+3
+              const uint32_t dst = stage_base + s * kSB;
+              if constexpr (kF8) {
+                tma_gather4(dst + kF8CodeOff + lane * 4 * 128, &maps.row, vcol0, r[0], r[1], r[2], r[3], fb);
+                tma_gather4(dst + kF8CodeOff + kF8CodeBoxBytes + lane * 4 * 128, &maps.row, vcol0 + 128, r[0], r[1],
+                            r[2], r[3], fb);
+                tma_gather4(dst + kRopeOff + lane * 4 * 64, &maps.rope_row, kF8RopeOff + 64 * (int)crank, r[0], r[1],
+                            r[2], r[3], fb);
+                tma_gather4(dst + kF8ScaleStageOff + lane * 128, &maps.scale_row, kF8ScaleOff, r[0], r[1], r[2], r[3],
                             fb);
-              tma_gather4(dst + kRopeOff + lane * 4 * 64, &maps.rope_row, rcol0, r[0], r[1], r[2], r[3], fb);
+              } else {
+#pragma unroll
+                for (int bx = 0; bx < kVBoxes; ++bx)
+                  tma_gather4(dst + bx * kBoxBytes + lane * 4 * 128, &maps.row, vcol0 + 64 * bx, r[0], r[1], r[2], r[3],
+                              fb);
+                tma_gather4(dst + kRopeOff + lane * 4 * 64, &maps.rope_row, rcol0, r[0], r[1], r[2], r[3], fb);
+              }
             }
+            __syncwarp();
+            ++k;
           }
-          __syncwarp();
         }
       }
     }
@@ -594,6 +664,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kF8 ? kThreadsF8 : k
             if (mbar_test_wait(smem_addr(kF8 ? &misc->conv_full[kk % kStages] : &misc->full[kk % kStages]),
                                (kk / kStages) & 1) &&
                 (kk < 2 || mbar_test_wait(smem_addr(&misc->s_free[kk & 1]), ((kk >> 1) & 1) ^ 1))) {
+              // gathered bf16 rows partly written by cp.async (generic proxy):
+              // order them before the tensor core's reads
+              if (!kF8 && a.topk > 0) fence_proxy_async_smem();
               tc_fence_after();
               // all 18 MMAs back to back: the tensor pipe overlaps dependent MMAs
               // only while they are queued together
@@ -883,12 +956,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kF8 ? kThreadsF8 : k
       return true;
     };
 
+    int js = 0;
     while (ok && cur.next(task, pg0, pg1, split)) {
       write_q(1);
       const int n = pg1 - pg0;
       for (int i = 0; ok && i < n; ++i) ok = send_s(k + i);
       if (!ok) break;
       k += n;
+      ++js;
     }
     if (ok && k > 0) ok = relay_read(k - 1);
     // the peer relays "slot read" for every score tile sent; collect the last one before exit

@@ -129,6 +129,16 @@ MLA_DEV void tma_gather4(uint32_t dst, const CUtensorMap* map, int32_t c0, int32
       : "memory");
 }
 
+// 16-byte asynchronous copy global -> shared (L2 only), and the arrive on an
+// mbarrier that fires once all of this thread's earlier cp.async copies have
+// landed (.noinc: the arrival counts toward the barrier's expected count).
+MLA_DEV void cp_async_16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+MLA_DEV void cp_async_arrive_noinc(uint32_t bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
+}
+
 // ---------------------------------------------------------------- DSMEM
 
 // 16-byte asynchronous store into another CTA's shared memory; completes 16
