@@ -253,6 +253,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kF8 ? kThreadsF8 : k
   Waiter W{misc, reinterpret_cast<uint32_t*>(a.plan + kPlanErr)};
 
   if (stage_base & 1023u) {  // cannot place the swizzled ring: refuse instead of corrupting
+    grid_dependency_wait();   // the plan kernel writes the error word too
     if (threadIdx.x == 0) atomicOr(W.err, kErrTimeout);
     return;
   }
@@ -298,6 +299,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kF8 ? kThreadsF8 : k
   cluster_sync();
   tc_fence_after();
   const uint32_t tmem = misc->tmem_base;
+  // Everything above overlaps the plan kernel (programmatic launch); the
+  // plan, q and the cache are read only after it has finished.
+  grid_dependency_wait();
   // Cache columns of this CTA: output columns [vcol0, vcol0 + 256) in four
   // 128-byte-swizzled boxes, and rope columns [rcol0, rcol0 + 32) in one
   // 64-byte-swizzled box; the scores are contracted over both (288 columns).
@@ -1083,6 +1087,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kF8 ? kThreadsF8 : k
   }
 
   // ------------------------------------------------------------ teardown
+  // The combine may launch once every CTA is here (its blocks then wait for
+  // the whole grid); triggering earlier would park them beside running CTAs.
+  allow_dependents();
   tc_fence_before();
   cluster_sync();  // no remote access to this CTA's shared memory after this point
   if (warp == 1) {
@@ -1101,13 +1108,23 @@ const void* decode_kernel_ptr(bool fp8) {
 int decode_smem_bytes(bool fp8) { return fp8 ? dec::smem_bytes<true>() : dec::smem_bytes<false>(); }
 int decode_threads(bool fp8) { return fp8 ? dec::kThreadsF8 : dec::kThreads; }
 
+// Launched with programmatic stream serialization: the CTAs start (barriers,
+// TMEM, cluster sync) while the plan kernel before them still runs, and wait
+// for it before reading anything it or earlier work produced.
 cudaError_t launch_decode(const CacheMaps& maps, const DecodeArgs& args, int workers, bool fp8,
                           cudaStream_t stream) {
-  if (fp8)
-    dec::mla_decode_kernel<true><<<2 * workers, dec::kThreadsF8, dec::smem_bytes<true>(), stream>>>(maps, args);
-  else
-    dec::mla_decode_kernel<false><<<2 * workers, dec::kThreads, dec::smem_bytes<false>(), stream>>>(maps, args);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * workers, 1, 1);
+  cfg.blockDim = dim3(fp8 ? dec::kThreadsF8 : dec::kThreads, 1, 1);
+  cfg.dynamicSmemBytes = fp8 ? dec::smem_bytes<true>() : dec::smem_bytes<false>();
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return fp8 ? cudaLaunchKernelEx(&cfg, dec::mla_decode_kernel<true>, maps, args)
+             : cudaLaunchKernelEx(&cfg, dec::mla_decode_kernel<false>, maps, args);
 }
 
 }  // namespace mla

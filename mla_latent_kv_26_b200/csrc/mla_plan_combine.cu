@@ -2,6 +2,7 @@
 #include <math.h>
 
 #include "common.cuh"
+#include "sm100.cuh"
 
 namespace mla {
 
@@ -10,7 +11,7 @@ namespace mla {
 // and ceil(ntok/64) pages; prefix[] lays the positions' pages end to end;
 // worker j of group g owns the group's pages [j*quota_g, (j+1)*quota_g).
 __global__ void __launch_bounds__(1024) mla_plan_kernel(PlanArgs a) {
-  __shared__ int s_scan[1024];
+  __shared__ int s_scan[32];
   __shared__ int s_carry;
   __shared__ unsigned s_err;
   const int tid = threadIdx.x;
@@ -38,17 +39,29 @@ __global__ void __launch_bounds__(1024) mla_plan_kernel(PlanArgs a) {
       ntok[t] = n;
       pages = (n + kPage - 1) / kPage;
     }
-    s_scan[tid] = pages;
-    __syncthreads();
-    for (int off = 1; off < 1024; off <<= 1) {
-      const int v = tid >= off ? s_scan[tid - off] : 0;
-      __syncthreads();
-      s_scan[tid] += v;
-      __syncthreads();
+    // inclusive scan: within each warp by shuffles, then over the 32 warp totals
+    const int lane = tid & 31, warp = tid >> 5;
+    int v = pages;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int n = __shfl_up_sync(~0u, v, off);
+      if (lane >= off) v += n;
     }
-    if (t < T) prefix[t] = s_carry + s_scan[tid] - pages;
+    if (lane == 31) s_scan[warp] = v;
     __syncthreads();
-    if (tid == 1023) s_carry += s_scan[1023];
+    if (warp == 0) {
+      int w = s_scan[lane];
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int n = __shfl_up_sync(~0u, w, off);
+        if (lane >= off) w += n;
+      }
+      s_scan[lane] = w;
+    }
+    __syncthreads();
+    if (t < T) prefix[t] = s_carry + (warp > 0 ? s_scan[warp - 1] : 0) + v - pages;
+    __syncthreads();
+    if (tid == 1023) s_carry += s_scan[31];
     __syncthreads();
   }
   if (tid == 0) {
@@ -74,6 +87,7 @@ __global__ void __launch_bounds__(1024) mla_plan_kernel(PlanArgs a) {
 // the worker), so each half merges with its own LSEs:
 // lse = M + ln sum_w exp(lse_w - M), out = sum_w exp(lse_w - lse) * o_w.
 __global__ void __launch_bounds__(256) mla_combine_kernel(CombineArgs a) {
+  ptx::grid_dependency_wait();  // the decode's partials (programmatic launch)
   const int T = a.plan[kPlanTasks];
   const int t = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -202,10 +216,19 @@ cudaError_t launch_plan(const PlanArgs& args, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
+// Launched with programmatic stream serialization behind the decode: its
+// blocks take SMs as decode CTAs finish and wait for the whole decode.
 cudaError_t launch_combine(const CombineArgs& args, int tasks, cudaStream_t stream) {
-  dim3 grid(tasks, (args.heads + 7) / 8);
-  mla_combine_kernel<<<grid, 256, 0, stream>>>(args);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(tasks, (args.heads + 7) / 8, 1);
+  cfg.blockDim = dim3(256, 1, 1);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, mla_combine_kernel, args);
 }
 
 }  // namespace mla

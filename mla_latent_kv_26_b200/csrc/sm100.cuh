@@ -139,6 +139,13 @@ MLA_DEV void cp_async_arrive_noinc(uint32_t bar) {
   asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
 }
 
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialization may start while the previous kernel in the stream runs;
+// grid_dependency_wait() returns once that kernel has completed and its
+// writes are visible. allow_dependents() lets the next such kernel launch.
+MLA_DEV void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+MLA_DEV void allow_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ---------------------------------------------------------------- DSMEM
 
 // 16-byte asynchronous store into another CTA's shared memory; completes 16
