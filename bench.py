@@ -770,6 +770,7 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle time for cpu_baseline")
     ap.add_argument("--profile", action="store_true", help="kernel launches only (for ncu): no e2e/oracle/clocks")
     ap.add_argument("--num-sms", type=int, default=0)
+    ap.add_argument("--e2e-lanes", type=int, default=4, help="decoders / streams the end-to-end steps rotate over")
     ap.add_argument("--op", default="decode", choices=["decode", "insert", "absorb", "indexer"],
                     help="decode: the decode step (default); insert: the latent-cache insert alone; "
                          "absorb: the absorb + un-absorb projections; indexer: fp8 index scores + top-k")
@@ -917,14 +918,20 @@ def main():
 
     # ---- end to end through the public API with pinned host buffers: every
     # step copies its inputs in and its output and LSE back. Consecutive steps
-    # alternate between two decoders on two streams, so one step's copies
-    # overlap the neighbouring steps' kernels (as a caller decoding step after
-    # step would run it); each stream keeps its own device buffers.
+    # rotate over --e2e-lanes decoders on as many streams, so one step's
+    # copies overlap the neighbouring steps' kernels (as a caller decoding
+    # step after step would run it); each stream keeps its own device
+    # buffers. A lane runs copy in -> kernels -> copy out in order, so with L
+    # lanes a step costs at least (copy in + kernels + copy out) / L: two
+    # lanes leave the step copy-bound on C3 (564 us against 401 us of
+    # kernels), three make it kernel-bound (393 us); small workloads, whose
+    # copies outweigh their kernels, still gain from a fourth (C5: 172, 109,
+    # 89 us).
     host_in = {k: inp[k].pin_memory() for k in ("q", "block_table", "seq_lens")}
     if inp["indices"] is not None:
         host_in["indices"] = inp["indices"].pin_memory()
     lanes = []
-    for li in range(2):
+    for li in range(max(1, args.e2e_lanes)):
         dl = dec if li == 0 else decoder_for(inp, num_sms=args.num_sms, device=dev)
         lanes.append({
             "dec": dl,
@@ -1037,7 +1044,7 @@ def main():
                 "h2d_bytes_per_step": acc["h2d_bytes"], "d2h_bytes_per_step": acc["d2h_bytes"],
                 "ms_per_step": e2e_ms, "streams": len(lanes),
                 "note": "plan + decode + combine through the C ABI, inputs from pinned host memory and out/lse "
-                        "back every step; consecutive steps alternate between two decoders on two streams"},
+                        f"back every step; consecutive steps rotate over {len(lanes)} decoders on as many streams"},
         "gpu_launches": 3 * K,
         "kernels_us": {"plan": plan_ms * 1e3, "decode": decode_ms * 1e3, "combine": combine_ms * 1e3,
                        "sampled_steps": len(kev), "statistic": "median of the sampled timed steps",
