@@ -18,8 +18,12 @@
 //               buffers when the group changes (128-byte swizzle, K-major)
 //   warp 1      tcgen05 issuer: D[128 keys, G*h] = K_tile . Q_group^T, four
 //               kind::f8f6f4 MMAs (K = 32 each) into one of two TMEM buffers
-//   warps 2-5   epilogue, one TMEM lane (key) per thread: ReLU, head weights,
-//               key scale, one fp32 score per (query, key), coalesced stores
+//   warps 2-9   epilogue, two groups of four warps taking alternate tiles
+//               (group g reads TMEM buffer g), one TMEM lane (key) per
+//               thread: ReLU, head weights, key scale, one fp32 score per
+//               (query, key), coalesced stores. With one group the epilogue
+//               set the pace (the kernel took 92.6 us against 55.8 us with
+//               the epilogue's arithmetic left out).
 //
 // mla_topk_kernel: one cluster of C CTAs (C = 1..8) per row; CTA c owns the
 // positions [c * chunk, (c + 1) * chunk) of the row, kept in shared memory
@@ -86,7 +90,7 @@ MLA_DEV uint32_t ld_shared_cluster_u32(uint32_t cluster_addr) {
   return v;
 }
 
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;   // producer, MMA issuer, 2 x 4 epilogue warps
 constexpr int kStages = 6;
 constexpr int kKeys = 128;                 // keys per tile: the MMA's M
 constexpr int kDim = 128;                  // index head width d: 128 fp8 = one 128-byte swizzle row
@@ -198,7 +202,7 @@ __global__ void __launch_bounds__(kThreads, 1) mla_index_kernel(const __grid_con
       mbar_init(smem_addr(&bars.q_full[i]), 1);
       mbar_init(smem_addr(&bars.q_empty[i]), 1);
       mbar_init(smem_addr(&bars.t_full[i]), 1);
-      mbar_init(smem_addr(&bars.t_empty[i]), 4);  // the four epilogue warps
+      mbar_init(smem_addr(&bars.t_empty[i]), 4);  // the four epilogue warps of group i
     }
     mbar_init(smem_addr(&bars.done), 1);
     bars.abort_flag = 0u;
@@ -278,21 +282,24 @@ __global__ void __launch_bounds__(kThreads, 1) mla_index_kernel(const __grid_con
   } else {
     // ------------------------------------------------------------ epilogue
     const int quad = warp & 3;
+    const int grp = (warp - 2) >> 2;   // tiles k with k % 2 == grp, TMEM buffer grp
     const int row = quad * 32 + lane;  // key within the tile = TMEM lane
     const uint32_t lanes = tmem + ((uint32_t)(quad * 32) << 16);
-    int k = 0;
-    // the key scale of the next item is loaded while this one is computed
+    int k = grp;
+    // the key scale of this group's next item is loaded while this one is computed
     auto key_scale = [&](const ItemCursor& c) -> float {
       const int t = c.j * kKeys + row;
       return t < a.n ? __ldg(a.k_s + (size_t)c.bb * a.n + t) : 0.f;
     };
-    float ks_next = i0 < i1 ? key_scale(cur) : 0.f;
-    for (long long it = i0; it < i1; ++it, ++k) {
-      const int tb = k & 1;
+    if (grp) cur.next();
+    float ks_next = i0 + grp < i1 ? key_scale(cur) : 0.f;
+    for (long long it = i0 + grp; it < i1; it += 2, k += 2) {
+      const int tb = grp;
       const ItemCursor c = cur;
       const float ks = ks_next;
       cur.next();
-      if (it + 1 < i1) ks_next = key_scale(cur);
+      cur.next();
+      if (it + 2 < i1) ks_next = key_scale(cur);
       if (!W.wait_warp(&bars.t_full[tb], (k >> 1) & 1)) break;
       tc_fence_after();
       const int bb = c.bb, g = c.g;
