@@ -18,10 +18,11 @@
 // same P for all 128 rows and accumulate their output halves with it.
 //
 // Per CTA (448 threads):
-//   warp 0      TMA producer: 64-token pages (block table) or 64 gathered rows
-//               (top-k indices, tile::gather4) into a 4-stage ring; a stage is
-//               four boxes of 64 rows x 128 B (128-byte swizzle) and one box
-//               of 64 rows x 64 B (64-byte swizzle)
+//   warp 0      producer: 64-token pages (block table, TMA) or 64 gathered
+//               rows (top-k indices; tile::gather4 for latent boxes 0-1 and
+//               the rope box, 16-byte cp.async for boxes 2-3) into a 4-stage
+//               ring; a stage is four boxes of 64 rows x 128 B (128-byte
+//               swizzle) and one box of 64 rows x 64 B (64-byte swizzle)
 //   warp 1      tcgen05 issuer: S = Q_slice * K_slice^T (M=128 heads, N=64
 //               tokens, K=288; A = Q in TMEM, its rope columns from shared
 //               memory) into one of two S buffers, and O += P * V (M=128,
