@@ -178,6 +178,34 @@ def test_split_invariance(dev):
     assert (l1 - l2).abs().max() < 1e-4
 
 
+def test_back_to_back_steps_with_changing_lengths(dev):
+    """Steps on one decoder and one stream with no host synchronisation
+    between them, the lengths (and so the plan and the split) changing every
+    step. The plan, decode and combine are chained as programmatic
+    dependents: a step's decode must read that step's plan, and must not
+    overwrite the previous step's partials before its combine has merged
+    them. Each step's result is copied on the same stream before the next
+    step starts writing."""
+    from mla_latent_kv_26_b200.workloads import small
+
+    steps = [[3000, 700, 64, 1], [1, 5000, 200, 129], [4097, 2, 3000, 65], [0, 64, 1, 2000]] * 2
+    cap = [max(col) for col in zip(*steps)]
+    d = small(batch=4, heads=128, lens=cap, seed=71)
+    g = _to(d, dev)
+    dec = run_gpu(d, dev)[4]
+    lens_dev = [torch.tensor(L, dtype=torch.int32, device=dev) for L in steps]
+    torch.cuda.synchronize(dev)
+    outs = []
+    for sl in lens_dev:
+        dec(g["q"], g["cache"], g["block_table"], sl)
+        outs.append((dec.out.clone(), dec.lse.clone()))
+    torch.cuda.synchronize(dev)
+    assert dec.error() == (0, 0)
+    for L, (o, l) in zip(steps, outs):
+        o_ref, l_ref = oracle.mla_decode(d["q"], d["cache"], d["block_table"], torch.tensor(L, dtype=torch.int32))
+        assert_parity(o.double().cpu(), l.double().cpu(), o_ref, l_ref, f"back-to-back {L}")
+
+
 def test_deterministic(dev):
     from mla_latent_kv_26_b200.workloads import small
 
