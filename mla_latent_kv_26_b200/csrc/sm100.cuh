@@ -366,6 +366,16 @@ MLA_DEV uint32_t pack_bf16x2(float lo, float hi) {
 // each product rounded to float32 and then to bf16: eight bf16 in a uint4.
 // The hardware widens two codes at a time to f16 (exact: every e4m3 value is
 // an f16 normal or zero), f16 -> float32 is exact, the product is one FMUL.
+// Both products of a pair come from one packed two-lane multiply
+// (mul.rn.f32x2: two IEEE round-to-nearest float32 products).
+MLA_DEV float2 mul2_rn(float2 a, float s) {
+  float2 d;
+  asm("{\n\t.reg .b64 pa, pb, pd;\n\tmov.b64 pa, {%2, %3};\n\tmov.b64 pb, {%4, %4};\n\t"
+      "mul.rn.f32x2 pd, pa, pb;\n\tmov.b64 {%0, %1}, pd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(s));
+  return d;
+}
 MLA_DEV uint4 dequant8_e4m3(uint32_t w0, uint32_t w1, float s) {
   const uint32_t w[2] = {w0, w1};
   uint32_t o[4];
@@ -374,8 +384,8 @@ MLA_DEV uint4 dequant8_e4m3(uint32_t w0, uint32_t w1, float s) {
 #pragma unroll
     for (int q = 0; q < 2; ++q) {
       const __nv_fp8x2_storage_t pair = (__nv_fp8x2_storage_t)((w[h] >> (16 * q)) & 0xFFFFu);
-      const float2 f = __half22float2(__half2(__nv_cvt_fp8x2_to_halfraw2(pair, __NV_E4M3)));
-      o[2 * h + q] = pack_bf16x2(__fmul_rn(f.x, s), __fmul_rn(f.y, s));
+      const float2 f = mul2_rn(__half22float2(__half2(__nv_cvt_fp8x2_to_halfraw2(pair, __NV_E4M3))), s);
+      o[2 * h + q] = pack_bf16x2(f.x, f.y);
     }
   }
   return make_uint4(o[0], o[1], o[2], o[3]);
