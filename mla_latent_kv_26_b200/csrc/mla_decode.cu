@@ -770,10 +770,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kF8 ? kThreadsF8 : k
           for (int c = 0; c < 8; ++c) {
             float v0, v1, v2, v3;
             fx23_unpack4(w[3 * c], w[3 * c + 1], w[3 * c + 2], inv, bias, v0, v1, v2, v3);
-            sc[4 * c + 0] = __uint_as_float(own[4 * c + 0]) + v0;
-            sc[4 * c + 1] = __uint_as_float(own[4 * c + 1]) + v1;
-            sc[4 * c + 2] = __uint_as_float(own[4 * c + 2]) + v2;
-            sc[4 * c + 3] = __uint_as_float(own[4 * c + 3]) + v3;
+            const float2 s01 = add2_rn(make_float2(__uint_as_float(own[4 * c + 0]), __uint_as_float(own[4 * c + 1])),
+                                       make_float2(v0, v1));
+            const float2 s23 = add2_rn(make_float2(__uint_as_float(own[4 * c + 2]), __uint_as_float(own[4 * c + 3])),
+                                       make_float2(v2, v3));
+            sc[4 * c + 0] = s01.x;
+            sc[4 * c + 1] = s01.y;
+            sc[4 * c + 2] = s23.x;
+            sc[4 * c + 3] = s23.y;
           }
         }
         __syncwarp();
@@ -807,21 +811,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kF8 ? kThreadsF8 : k
           corr = i > 0;
         }
         const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
-        const float sl2 = a.scale_log2;
+        const float2 sl2 = make_float2(a.scale_log2, a.scale_log2), nm = make_float2(-m_use, -m_use);
         uint32_t pp[16];
-        float ps[16];
+        float2 ps[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+        // two scores per packed instruction: the exponent arguments and the
+        // row sum (four packed accumulators)
 #pragma unroll
         for (int c = 0; c < 16; ++c) {
-          const float p0 = ex2(fmaf(sc[2 * c], sl2, -m_use));
-          const float p1 = ex2(fmaf(sc[2 * c + 1], sl2, -m_use));
-          pp[c] = pack_bf16x2(p0, p1);
-          ps[c] = p0 + p1;
+          const float2 e = fma2_rn(make_float2(sc[2 * c], sc[2 * c + 1]), sl2, nm);
+          const float2 p = make_float2(ex2(e.x), ex2(e.y));
+          pp[c] = pack_bf16x2(p.x, p.y);
+          ps[c & 3] = add2_rn(ps[c & 3], p);
         }
-#pragma unroll
-        for (int c = 0; c < 8; ++c) ps[c] += ps[c + 8];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) ps[c] += ps[c + 4];
-        l_run += (ps[0] + ps[2]) + (ps[1] + ps[3]);
+        ps[0] = add2_rn(ps[0], ps[2]);
+        ps[1] = add2_rn(ps[1], ps[3]);
+        ps[0] = add2_rn(ps[0], ps[1]);
+        l_run += ps[0].x + ps[0].y;
         const float l_row = l_run + __shfl_xor_sync(~0u, l_run, 16);
 
         // P buffer xs is free once both CTAs' PV of tile k-2 completed

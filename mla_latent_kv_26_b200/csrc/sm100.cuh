@@ -376,6 +376,24 @@ MLA_DEV float2 mul2_rn(float2 a, float s) {
       : "f"(a.x), "f"(a.y), "f"(s));
   return d;
 }
+// a + b and a * b + c on two float32 lanes at once (add.rn.f32x2 /
+// fma.rn.f32x2: the same IEEE results as two FADD / FFMA).
+MLA_DEV float2 add2_rn(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 pa, pb, pd;\n\tmov.b64 pa, {%2, %3};\n\tmov.b64 pb, {%4, %5};\n\t"
+      "add.rn.f32x2 pd, pa, pb;\n\tmov.b64 {%0, %1}, pd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+MLA_DEV float2 fma2_rn(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{\n\t.reg .b64 pa, pb, pc, pd;\n\tmov.b64 pa, {%2, %3};\n\tmov.b64 pb, {%4, %5};\n\t"
+      "mov.b64 pc, {%6, %7};\n\tfma.rn.f32x2 pd, pa, pb, pc;\n\tmov.b64 {%0, %1}, pd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
 MLA_DEV uint4 dequant8_e4m3(uint32_t w0, uint32_t w1, float s) {
   const uint32_t w[2] = {w0, w1};
   uint32_t o[4];
