@@ -941,10 +941,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kF8 ? kThreadsF8 : k
       const float mult = fx23_mult(ex);
       uint32_t w[24];
 #pragma unroll
-      for (int c = 0; c < 8; ++c)
-        fx23_pack4(fx23_code(__uint_as_float(sr[4 * c]), mult), fx23_code(__uint_as_float(sr[4 * c + 1]), mult),
-                   fx23_code(__uint_as_float(sr[4 * c + 2]), mult), fx23_code(__uint_as_float(sr[4 * c + 3]), mult),
-                   w[3 * c], w[3 * c + 1], w[3 * c + 2]);
+      for (int c = 0; c < 8; ++c) {
+        uint32_t c0, c1, c2, c3;
+        fx23_code2(__uint_as_float(sr[4 * c]), __uint_as_float(sr[4 * c + 1]), mult, c0, c1);
+        fx23_code2(__uint_as_float(sr[4 * c + 2]), __uint_as_float(sr[4 * c + 3]), mult, c2, c3);
+        fx23_pack4(c0, c1, c2, c3, w[3 * c], w[3 * c + 1], w[3 * c + 2]);
+      }
       // the peer's softmax warps have read its slot for tile kk - kXSlots (so
       // that copy has also finished reading this CTA's staging buffer)
       const int xs = kk % kXSlots;

@@ -349,12 +349,7 @@ MLA_DEV float fx23_val(uint32_t bits24, float inv, float bias) {
 }
 // Three words -> four values.
 MLA_DEV void fx23_unpack4(uint32_t w0, uint32_t w1, uint32_t w2, float inv, float bias, float& v0, float& v1,
-                          float& v2, float& v3) {
-  v0 = fx23_val(w0, inv, bias);
-  v1 = fx23_val(__byte_perm(w0, w1, 0x0543), inv, bias);
-  v2 = fx23_val(__byte_perm(w1, w2, 0x0432), inv, bias);
-  v3 = fx23_val(w2 >> 8, inv, bias);
-}
+                          float& v2, float& v3);
 
 // Two floats -> bf16x2 (round to nearest even), `lo` in the low half.
 MLA_DEV uint32_t pack_bf16x2(float lo, float hi) {
@@ -393,6 +388,25 @@ MLA_DEV float2 fma2_rn(float2 a, float2 b, float2 c) {
       : "=f"(d.x), "=f"(d.y)
       : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
   return d;
+}
+// Three words -> four values, the FMAs two lanes at a time.
+MLA_DEV void fx23_unpack4(uint32_t w0, uint32_t w1, uint32_t w2, float inv, float bias, float& v0, float& v1,
+                          float& v2, float& v3) {
+  const auto f = [](uint32_t bits24) { return __uint_as_float((bits24 & 0x00FFFFFFu) | 0x4B000000u); };
+  const float2 ib = make_float2(inv, inv), bb = make_float2(bias, bias);
+  const float2 a = fma2_rn(make_float2(f(w0), f(__byte_perm(w0, w1, 0x0543))), ib, bb);
+  const float2 b = fma2_rn(make_float2(f(__byte_perm(w1, w2, 0x0432)), f(w2 >> 8)), ib, bb);
+  v0 = a.x;
+  v1 = a.y;
+  v2 = b.x;
+  v3 = b.y;
+}
+// Two codes at a time: the FMAs of fx23_code on two lanes, then the clamps.
+MLA_DEV void fx23_code2(float x0, float x1, float mult, uint32_t& c0, uint32_t& c1) {
+  constexpr float kMagic = 12582912.0f, kLo = kMagic - 4194303.0f, kHi = kMagic + 4194303.0f;
+  const float2 y = fma2_rn(make_float2(x0, x1), make_float2(mult, mult), make_float2(kMagic, kMagic));
+  c0 = __float_as_uint(fminf(fmaxf(y.x, kLo), kHi));
+  c1 = __float_as_uint(fminf(fmaxf(y.y, kLo), kHi));
 }
 MLA_DEV uint4 dequant8_e4m3(uint32_t w0, uint32_t w1, float s) {
   const uint32_t w[2] = {w0, w1};
