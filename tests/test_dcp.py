@@ -87,7 +87,9 @@ def _rank_main(rank, world, port, name, q):
         out, lse = dcp_decode(d["q"], d["cache"], d["block_table"], d["seq_lens"], world=world, rank=rank,
                               q_len=d["q_len"], causal=d["causal"], indices=d["indices"],
                               decode=_oracle_decode, merge=_oracle_merge)
-        q.put((rank, out, lse))
+        # by value (numpy): a tensor would travel as a file descriptor that the
+        # parent fetches from this process, which may have exited by then
+        q.put((rank, out.numpy(), lse.numpy()))
     finally:
         dist.destroy_process_group()
 
@@ -111,6 +113,7 @@ def test_dcp_gloo_ranks_match_unsharded_oracle(world, name):
     o_ref, l_ref = oracle.mla_decode(d["q"], d["cache"], d["block_table"], d["seq_lens"], causal=d["causal"],
                                      indices=d["indices"])
     for rank, out, lse in results:
+        out, lse = torch.from_numpy(out), torch.from_numpy(lse)
         # each rank's partial travelled as float32: agreement to float32 rounding
         assert torch.allclose(out, o_ref, rtol=1e-5, atol=1e-5), (name, rank)
         fin = torch.isfinite(l_ref)
