@@ -933,9 +933,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kF8 ? kThreadsF8 : k
       if (!W.wait_warp(&misc->full[s], (kk / kStages) & 1)) return false;
       const uint32_t msk = (uint32_t)(misc->stage_mask[s] >> (32 * th));
       float amax = 0.f;
+      if (msk == ~0u) {  // every token valid (the common case): a max tree, no bit tests
+        float t[16];
 #pragma unroll
-      for (int c = 0; c < 32; ++c)
-        if ((msk >> c) & 1u) amax = fmaxf(amax, fabsf(__uint_as_float(sr[c])));
+        for (int c = 0; c < 16; ++c) t[c] = fmaxf(fabsf(__uint_as_float(sr[c])), fabsf(__uint_as_float(sr[c + 16])));
+#pragma unroll
+        for (int c = 0; c < 8; ++c) t[c] = fmaxf(t[c], t[c + 8]);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) t[c] = fmaxf(t[c], t[c + 4]);
+        amax = fmaxf(fmaxf(t[0], t[2]), fmaxf(t[1], t[3]));
+      } else {
+#pragma unroll
+        for (int c = 0; c < 32; ++c)
+          if ((msk >> c) & 1u) amax = fmaxf(amax, fabsf(__uint_as_float(sr[c])));
+      }
       amax = fmaxf(amax, __shfl_xor_sync(~0u, amax, 16));
       const uint32_t ex = fx23_exponent(amax);
       const float mult = fx23_mult(ex);
