@@ -948,7 +948,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kF8 ? kThreadsF8 : k
           if ((msk >> c) & 1u) amax = fmaxf(amax, fabsf(__uint_as_float(sr[c])));
       }
       amax = fmaxf(amax, __shfl_xor_sync(~0u, amax, 16));
-      const uint32_t ex = fx23_exponent(amax);
+      const uint32_t ex = fx23_exponent(fx23_headroom(amax));
       const float mult = fx23_mult(ex);
       uint32_t w[24];
 #pragma unroll

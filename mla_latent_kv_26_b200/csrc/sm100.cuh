@@ -401,13 +401,20 @@ MLA_DEV void fx23_unpack4(uint32_t w0, uint32_t w1, uint32_t w2, float inv, floa
   v2 = b.x;
   v3 = b.y;
 }
-// Two codes at a time: the FMAs of fx23_code on two lanes, then the clamps.
+// Two codes at a time, the FMAs on two lanes and no clamp: with the row's
+// exponent taken from fx23_headroom(max|x|), every |x| <= max|x| gives
+// |round(x * mult)| <= 2^22 - 1. (Values outside that range - masked
+// tokens, which the receiver discards - stay inside their own 3-byte field.)
 MLA_DEV void fx23_code2(float x0, float x1, float mult, uint32_t& c0, uint32_t& c1) {
-  constexpr float kMagic = 12582912.0f, kLo = kMagic - 4194303.0f, kHi = kMagic + 4194303.0f;
+  constexpr float kMagic = 12582912.0f;
   const float2 y = fma2_rn(make_float2(x0, x1), make_float2(mult, mult), make_float2(kMagic, kMagic));
-  c0 = __float_as_uint(fminf(fmaxf(y.x, kLo), kHi));
-  c1 = __float_as_uint(fminf(fmaxf(y.y, kLo), kHi));
+  c0 = __float_as_uint(y.x);
+  c1 = __float_as_uint(y.y);
 }
+// max|x| * (1 + 2^-22): the exponent then leaves half a unit of headroom
+// below 2^22 (only rows whose maximum lies in the top 2^-22 of its binade
+// move to the next exponent).
+MLA_DEV float fx23_headroom(float amax) { return amax * 1.0000002384185791f; }
 MLA_DEV uint4 dequant8_e4m3(uint32_t w0, uint32_t w1, float s) {
   const uint32_t w[2] = {w0, w1};
   uint32_t o[4];
