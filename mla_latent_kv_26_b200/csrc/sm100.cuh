@@ -329,12 +329,6 @@ MLA_DEV float ex2(float x) {
 MLA_DEV uint32_t fx23_exponent(float amax) { return max((__float_as_uint(amax) >> 23) & 0xFFu, 22u); }
 MLA_DEV float fx23_mult(uint32_t e) { return __uint_as_float((275u - e) << 23); }  // 2^(148 - e)
 MLA_DEV float fx23_inv(uint32_t e) { return __uint_as_float((e - 21u) << 23); }    // 2^(e - 148)
-// x * mult + 1.5 * 2^23 has unit spacing: its low 23 bits are round(x mult) + 2^22
-// (bit 23, the exponent's lowest bit, is 0 over the clamped range).
-MLA_DEV uint32_t fx23_code(float x, float mult) {
-  constexpr float kMagic = 12582912.0f, kLo = kMagic - 4194303.0f, kHi = kMagic + 4194303.0f;
-  return __float_as_uint(fminf(fmaxf(fmaf(x, mult, kMagic), kLo), kHi));
-}
 // Four codes (low three bytes of each) -> three words.
 MLA_DEV void fx23_pack4(uint32_t c0, uint32_t c1, uint32_t c2, uint32_t c3, uint32_t& w0, uint32_t& w1, uint32_t& w2) {
   w0 = __byte_perm(c0, c1, 0x4210);
@@ -344,9 +338,6 @@ MLA_DEV void fx23_pack4(uint32_t c0, uint32_t c1, uint32_t c2, uint32_t c3, uint
 // q * inv from a 23-bit field u: 2^23 + u is rebuilt as float bits, and
 // (2^23 + u) * inv - (2^23 + 2^22) * inv is exact in one FMA.
 MLA_DEV float fx23_bias(float inv) { return -12582912.0f * inv; }
-MLA_DEV float fx23_val(uint32_t bits24, float inv, float bias) {
-  return fmaf(__uint_as_float((bits24 & 0x00FFFFFFu) | 0x4B000000u), inv, bias);
-}
 // Three words -> four values.
 MLA_DEV void fx23_unpack4(uint32_t w0, uint32_t w1, uint32_t w2, float inv, float bias, float& v0, float& v1,
                           float& v2, float& v3);
@@ -401,9 +392,11 @@ MLA_DEV void fx23_unpack4(uint32_t w0, uint32_t w1, uint32_t w2, float inv, floa
   v2 = b.x;
   v3 = b.y;
 }
-// Two codes at a time, the FMAs on two lanes and no clamp: with the row's
-// exponent taken from fx23_headroom(max|x|), every |x| <= max|x| gives
-// |round(x * mult)| <= 2^22 - 1. (Values outside that range - masked
+// x * mult + 1.5 * 2^23 has unit spacing: its low 23 bits are
+// round(x mult) + 2^22 (bit 23, the exponent's lowest bit, is 0 while
+// |round(x mult)| < 2^22). Two codes at a time, the FMAs on two lanes and no
+// clamp: with the row's exponent taken from fx23_headroom(max|x|), every
+// |x| <= max|x| gives |round(x * mult)| <= 2^22 - 1. (Values outside that range - masked
 // tokens, which the receiver discards - stay inside their own 3-byte field.)
 MLA_DEV void fx23_code2(float x0, float x1, float mult, uint32_t& c0, uint32_t& c1) {
   constexpr float kMagic = 12582912.0f;
