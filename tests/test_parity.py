@@ -335,9 +335,9 @@ def test_full_size_workload(dev, key):
 @pytest.mark.parametrize("heads", [128, 16])
 def test_large_magnitude_queries(dev, q_std, heads):
     """Queries 10x and 20x the usual scale against an N(0, 1) cache: partial
-    scores of each CTA half reach the hundreds, where the 16-bit block
+    scores of each CTA half reach the hundreds, where the 23-bit block
     fixed-point exchange of partial scores is coarsest (its error per score is
-    at most 2^-15 of the largest partial score of the row in the tile). Both
+    at most 2^-22 of the largest partial score of the row in the tile). Both
     the output and the LSE must stay within the usual tolerances."""
     from mla_latent_kv_26_b200.workloads import small
 

@@ -125,21 +125,25 @@ def test_fp8_decode_matches_oracle(libmla, dev, name, num_sms):
     assert torch.isfinite(out.float()).all()
 
 
-def test_fp8_decode_full_size_v3_shape(libmla, dev):
-    """The batch-64, 128-head, ragged 1k-32k workload over an fp8 cache, every
-    sequence against the oracle."""
+@pytest.mark.parametrize("key", ["C1", "C2", "C3", "C4", "C5"])
+def test_fp8_decode_full_size_workload(libmla, dev, key):
+    """The benchmark workloads at full size over an fp8 cache, in the
+    benchmark's launch configuration (all SMs): every sequence of the batch
+    against the oracle, the relative L2 error over the whole output."""
     from mla_latent_kv_26_b200.decoder import decoder_for
     from mla_latent_kv_26_b200.workloads import make_fp8_cache, make_inputs
 
-    d = make_inputs("C3")
+    d = make_inputs(key)
     raw = make_fp8_cache(d)
     del d["cache"]
     g = _to(d, dev)
     dec = decoder_for(d, device=dev)
-    out, lse = dec(g["q"], raw.to(dev), g["block_table"], g["seq_lens"])
+    out, lse = dec(g["q"], raw.to(dev), g["block_table"], g["seq_lens"], g["indices"])
     assert dec.error() == (0, 0)
-    o_ref, l_ref = oracle.mla_decode(d["q"], oracle.dequantize_cache(raw), d["block_table"], d["seq_lens"])
-    _assert_parity(out, lse, o_ref, l_ref, "fp8 C3")
+    assert torch.isfinite(out.float()).all() and torch.isfinite(lse).all()
+    o_ref, l_ref = oracle.mla_decode(d["q"], oracle.dequantize_cache(raw), d["block_table"], d["seq_lens"],
+                                     causal=d["causal"], indices=d["indices"])
+    _assert_parity(out, lse, o_ref, l_ref, f"fp8 {key}")
 
 
 def test_fp8_insert_then_decode_chain(libmla, dev):
