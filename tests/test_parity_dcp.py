@@ -34,30 +34,55 @@ def _parity(out, lse, o_ref, l_ref):
         assert float((lse[fin] - l_ref[fin]).abs().max()) <= 1e-3
 
 
-@pytest.mark.parametrize("world", [2, 3, 4])
-@pytest.mark.parametrize("case", ["dense", "causal", "sparse"])
-def test_dcp_emulated_ranks_match_oracle(libmla, dev, world, case):
+def _emulated_dcp(d, cache, world, dev):
+    """Every rank's shard decoded by the library one after another on one
+    GPU, then merged by mla_merge."""
     from mla_latent_kv_26_b200.dcp import _library_decode, library_merge, shard_inputs
-    from mla_latent_kv_26_b200.workloads import small
+
+    g = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in d.items() if k != "cache"}
+    cache = cache.to(dev)
+    outs, lses = [], []
+    for r in range(world):
+        shard = shard_inputs(g["block_table"], g["seq_lens"], world=world, rank=r, q_len=d["q_len"],
+                             causal=d["causal"], indices=g["indices"])
+        o, l = _library_decode(g["q"], cache, shard)
+        outs.append(o)
+        lses.append(l)
+    out, lse = library_merge(torch.stack(outs), torch.stack(lses))
+    torch.cuda.synchronize(dev)
+    return out, lse
+
+
+@pytest.mark.parametrize("world", [2, 3, 4])
+@pytest.mark.parametrize("case", ["dense", "causal", "sparse", "fp8"])
+def test_dcp_emulated_ranks_match_oracle(libmla, dev, world, case):
+    from mla_latent_kv_26_b200.workloads import make_fp8_cache, small
 
     if case == "dense":
         d = small(batch=4, heads=128, lens=[5000, 700, 1, 64], seed=31, nan_tail=True)
     elif case == "causal":
         d = small(batch=3, heads=128, q_len=2, causal=True, lens=[4097, 2, 130], seed=32)
-    else:
+    elif case == "sparse":
         d = small(batch=3, heads=128, lens=[9000, 300, 2100], topk=512, seed=33)
-    g = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in d.items()}
-    outs, lses = [], []
-    for r in range(world):
-        shard = shard_inputs(g["block_table"], g["seq_lens"], world=world, rank=r, q_len=d["q_len"],
-                             causal=d["causal"], indices=g["indices"])
-        o, l = _library_decode(g["q"], g["cache"], shard)
-        outs.append(o)
-        lses.append(l)
-    out, lse = library_merge(torch.stack(outs), torch.stack(lses))
-    torch.cuda.synchronize(dev)
-    o_ref, l_ref = oracle.mla_decode(d["q"], d["cache"], d["block_table"], d["seq_lens"], causal=d["causal"],
+    else:
+        d = small(batch=4, heads=128, lens=[6000, 129, 1, 700], seed=34)
+    cache = make_fp8_cache(d, nan_tail=True) if case == "fp8" else d["cache"]
+    out, lse = _emulated_dcp(d, cache, world, dev)
+    ref_cache = oracle.dequantize_cache(cache) if case == "fp8" else d["cache"]
+    o_ref, l_ref = oracle.mla_decode(d["q"], ref_cache, d["block_table"], d["seq_lens"], causal=d["causal"],
                                      indices=d["indices"])
+    _parity(out, lse, o_ref, l_ref)
+
+
+def test_dcp_full_size_workload_eight_ranks(libmla, dev):
+    """The batch-64, 128-head, ragged 1k-32k workload sharded over 8 emulated
+    ranks: every sequence of the merged result against the oracle's
+    un-sharded decode."""
+    from mla_latent_kv_26_b200.workloads import make_inputs
+
+    d = make_inputs("C3")
+    out, lse = _emulated_dcp(d, d["cache"], 8, dev)
+    o_ref, l_ref = oracle.mla_decode(d["q"], d["cache"], d["block_table"], d["seq_lens"])
     _parity(out, lse, o_ref, l_ref)
 
 

@@ -146,6 +146,37 @@ def test_fp8_decode_full_size_workload(libmla, dev, key):
     _assert_parity(out, lse, o_ref, l_ref, f"fp8 {key}")
 
 
+def test_fp8_cuda_graph_replay_with_new_lengths(libmla, dev):
+    """One captured step (plan, decode, combine over an fp8 cache) replayed
+    after the device-side lengths were changed in place: the plan runs inside
+    the graph, so the replay decodes the new lengths."""
+    from mla_latent_kv_26_b200.decoder import decoder_for
+    from mla_latent_kv_26_b200.workloads import make_fp8_cache, small
+
+    d = small(batch=3, heads=128, lens=[3000, 300, 64], seed=57)
+    raw = make_fp8_cache(d)
+    g = _to(d, dev)
+    cache = raw.to(dev)
+    dec = decoder_for(d, device=dev)
+    dec(g["q"], cache, g["block_table"], g["seq_lens"])
+    s = torch.cuda.Stream(dev)
+    s.wait_stream(torch.cuda.current_stream(dev))
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(graph, stream=s):
+            dec(g["q"], cache, g["block_table"], g["seq_lens"], stream=s)
+    torch.cuda.current_stream(dev).wait_stream(s)
+    # within each sequence's own pages: 3000 -> 3008 fills its last page,
+    # 300 -> 1 and 64 -> 0 shorten
+    new = torch.tensor([3008, 1, 0], dtype=torch.int32)
+    g["seq_lens"].copy_(new.to(dev))
+    graph.replay()
+    torch.cuda.synchronize(dev)
+    assert dec.error() == (0, 0)
+    o_ref, l_ref = oracle.mla_decode(d["q"], oracle.dequantize_cache(raw), d["block_table"], new)
+    _assert_parity(dec.out, dec.lse, o_ref, l_ref, "fp8 graph replay, new lengths")
+
+
 def test_fp8_insert_then_decode_chain(libmla, dev):
     """Insert new tokens into an fp8 cache on the GPU, decode over it on the
     GPU; the oracle inserts into a bf16 cache, quantises and decodes."""
