@@ -46,7 +46,7 @@ def _assert_parity(out, lse, o_ref, l_ref, where):
 # ---------------------------------------------------------------- insert
 
 
-@pytest.mark.parametrize("case", ["prefill", "decode-token", "zero-latent", "large-and-small"])
+@pytest.mark.parametrize("case", ["prefill", "decode-token", "zero-latent", "large-and-small", "prefill-64x1024"])
 def test_fp8_insert_codes_bit_exact(libmla, dev, case):
     from mla_latent_kv_26_b200.decoder import cache_insert
     from mla_latent_kv_26_b200.workloads import insert_inputs
@@ -55,6 +55,8 @@ def test_fp8_insert_codes_bit_exact(libmla, dev, case):
         d = insert_inputs(lens=[200, 70], new_tokens=[200, 70], seed=41)
     elif case == "decode-token":
         d = insert_inputs(lens=[300, 65, 1], new_tokens=[1, 1, 1], seed=42)
+    elif case == "prefill-64x1024":
+        d = insert_inputs(lens=[1024] * 64, new_tokens=[1024] * 64, seed=5)
     elif case == "zero-latent":
         d = insert_inputs(lens=[64], new_tokens=[64], seed=43)
         d["kv"][:5, :512] = 0

@@ -88,6 +88,14 @@ def test_insert_decode_batch_of_64(libmla, dev):
     assert err == 0
 
 
+def test_insert_full_size_prefill_64x1024(libmla, dev):
+    """The benchmark's insert workload: 64 sequences x 1,024 new tokens
+    (positions 0..1023, seed 5), every row against the oracle."""
+    d = insert_inputs(lens=[1024] * 64, new_tokens=[1024] * 64, seed=5)
+    err, skipped = check_full(libmla, d, dev, where="prefill 64x1024")
+    assert err == 0 and len(skipped) == 0
+
+
 def test_insert_scale_extremes_and_zero_row(libmla, dev):
     """Rows scaled by 2^-56 and 2^+56 (the float32 sum of squares of 512
     N(0,1) values times 2^112 stays far below the float32 maximum 2^128), and
